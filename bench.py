@@ -1,0 +1,466 @@
+#!/usr/bin/env python
+"""Benchmark of the ReSpinQuant block-boundary hot path on B200.
+
+One step = the whole path on one batch of tokens: the fused boundary kernel
+(rank-r basis fix + per-token INT4 quantization, ReSpinQuant explainers zh
+§2.2 and §3-§4) followed by the tcgen05 W4A4 GEMM that consumes its codes.
+Workload: Llama-2-7B-shaped, D = 4096, 2048 tokens per GPU, r = 32 (rank-64
+skew deviation, norm 0.1, 8 outlier channels x50), GEMM 4096 -> 11008 with
+INT4 weights uniform in [-8, 7]. Synthetic, seeded inputs.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun each rank processes its own 2048 tokens (weak scaling, no
+data-path collective); the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "tokens/s fused ΔT-lowrank+INT4 quant (D=4096,r=32); W4A4 GEMM TOPS"
+WORKLOAD = "llama2_7b"
+NSETS = 4            # rotating input sets: 4 x 56 MB > 126 MB L2
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+INT8_OVER_BF16 = 2.0  # nominal dense ratio (4.5 / 2.25 PFLOP/s)
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--profile-launch", choices=["boundary", "gemm"],
+                   help="profiling aid: warm up, then launch one kernel once "
+                        "(for ncu captures); prints no bench line")
+    p.add_argument("--tokens", type=int, default=None,
+                   help="tokens for --profile-launch (default 2048)")
+    return p.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            m = json.load(fh)
+        return float(m["hbm_gbs"]), float(m["bf16_tflops"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
+
+
+# ---------------------------------------------------------------- clocks
+
+REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting",
+           0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x10: "sync_boost",
+           0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+           0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+
+class ClockSampler(threading.Thread):
+    """Polls NVML (read only) for SM clock, throttle reasons and power."""
+
+    def __init__(self, torch_device: int, period_s: float = 0.005):
+        super().__init__(daemon=True)
+        self.period = period_s
+        self.samples = []
+        self.stop_evt = threading.Event()
+        self.ok = False
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            pr = torch.cuda.get_device_properties(torch_device)
+            bus = "%08x:%02x:%02x.0" % (pr.pci_domain_id, pr.pci_bus_id,
+                                        pr.pci_device_id)
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(
+                self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # pragma: no cover - depends on the box
+            self.err = repr(e)
+
+    def run(self):
+        if not self.ok:
+            return
+        nv = self.nv
+        while not self.stop_evt.is_set():
+            try:
+                t = time.time()
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                try:
+                    rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                except Exception:
+                    rs = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+                self.samples.append((t, mhz, rs))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def summary(self, t0: float, t1: float):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [],
+                    "samples": 0, "note": getattr(self, "err", "nvml")}
+        win = [s for s in self.samples if t0 <= s[0] <= t1]
+        if not win:   # region shorter than the poll period: nearest samples
+            win = sorted(self.samples, key=lambda s: abs(s[0] - t1))[:2]
+        mhz = sorted(s[1] for s in win)
+        mask = 0
+        for s in win:
+            mask |= s[2]
+        reasons = [n for b, n in REASONS.items() if mask & b and b != 0x1]
+        return {"sm_mhz": mhz[len(mhz) // 2] if mhz else None,
+                "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(win)}
+
+
+# ---------------------------------------------------------------- oracle legs
+
+def oracle_sample_rate(fx, qw, sw, n_boundary: int, n_gemm: int):
+    """Time the CPU oracle (as it stands) on a bounded sample; tokens/s of
+    the whole path per token = 1 / (t_boundary/token + t_gemm/token)."""
+    import numpy as np
+    from threadpoolctl import threadpool_limits
+
+    import oracle as O
+    with threadpool_limits(limits=1):
+        x = fx.x[:n_boundary].float().numpy()
+        res = fx.residual[:n_boundary].float().numpy()
+        U32, V32 = fx.U.astype(np.float32), fx.V.astype(np.float32)
+        t0 = time.perf_counter()
+        _, _, codes, scale = O.boundary_reference(x, res, U32, V32)
+        t1 = time.perf_counter()
+        qa = O.pack_int4(codes[:n_gemm])
+        acc = O.w4a4_acc(qa, qw)
+        O.w4a4_epilogue_bits(acc, scale[:n_gemm], sw)
+        t2 = time.perf_counter()
+    per_tok = (t1 - t0) / n_boundary + (t2 - t1) / n_gemm
+    return 1.0 / per_tok, (t2 - t0)
+
+
+def cpu_baseline_block(fx, qw, sw):
+    rate, secs = oracle_sample_rate(fx, qw, sw, 512, 32)
+    return {"value": rate, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": "boundary oracle (fp64 fix + binary32 quantizer) on 512 "
+                      "of the 2048 tokens, W4A4 GEMM oracle (exact int64 + "
+                      "binary32 epilogue) on 32 of the 2048 rows x 11008 "
+                      "channels; per-token times summed; %.1f s of CPU work, "
+                      "1 thread" % secs}
+
+
+def workload_inputs(device: str | None):
+    import numpy as np
+    import workloads as W
+    w = W.WORKLOADS[WORKLOAD]
+    fx = W.workload_fixture(WORKLOAD)
+    K = w.D
+    qw = W.int4_packed_random(w.O, K, 0, W.TID_WEIGHTS)
+    sw = W.weight_scales(w.O, K, 0)
+    return w, fx, qw, sw
+
+
+def run_reference(args, rank: int):
+    """The reference arm: the CPU oracle, timed on the host cores."""
+    if rank != 0:
+        return
+    w, fx, qw, sw = workload_inputs(None)
+    nb, ng = 64, 4
+    for _ in range(max(0, args.warmup)):
+        oracle_sample_rate(fx, qw, sw, nb, ng)
+    t = 0.0
+    rates = []
+    for _ in range(args.steps):
+        r, s = oracle_sample_rate(fx, qw, sw, nb, ng)
+        rates.append(r)
+        t += s
+    # per step: the full 2048-token batch at the sampled per-token cost
+    per_tok = sum(1.0 / r for r in rates) / len(rates)
+    value = 1.0 / per_tok
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value,
+        "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": per_tok * w.N * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64+f32+int64", "data": "synthetic",
+        "config": config_block(w, args.gpus),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1,
+                         "kind": "oracle",
+                         "sample": "each step: boundary oracle on 64 tokens "
+                                   "+ GEMM oracle on 4 rows, 1 thread; "
+                                   "%.1f s total" % t},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def config_block(w, n_gpus):
+    return {"workload": "Llama-2-7B-shaped boundary + W4A4 GEMM: D=4096, "
+                        "2048 tokens/GPU, r=32, GEMM 4096->11008",
+            "D": w.D, "tokens_per_gpu": w.N, "r": w.r, "gemm_out": w.O,
+            "global_batch": w.N * n_gpus, "parallelism": "dp%d" % n_gpus,
+            "l2": "inputs larger than L2: %d rotating input sets of %.0f MB"
+                  % (NSETS, (2 * w.N * w.D * 2 + w.O * w.D // 2) / 1e6)}
+
+
+def traffic_for(kernel_file: str, name: str):
+    """ncu DRAM bytes per launch recorded for this exact kernel source, or
+    None when the kernel changed since the capture."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    src = os.path.join(ROOT, "rotation_post_quantization_b200", "csrc",
+                       kernel_file)
+    try:
+        with open(path) as fh:
+            rec = json.load(fh).get(name)
+        with open(src, "rb") as fh:
+            sha = hashlib.sha256(fh.read()).hexdigest()
+        if rec and rec.get("source_sha256") == sha:
+            return rec["bytes_per_launch"]
+    except Exception:
+        pass
+    return None
+
+
+# ---------------------------------------------------------------- our arm
+
+def run_ours(args, rank: int, world: int, local_rank: int):
+    import numpy as np
+    import torch
+    import rotation_post_quantization_b200 as rq
+    import workloads as W
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        import datetime
+        dist.init_process_group("nccl", device_id=dev,
+                                timeout=datetime.timedelta(seconds=120))
+
+    w, fx, qw_np, sw_np = workload_inputs("cuda")
+    D, N, r, O_ = w.D, w.N, w.r, w.O
+    K = D
+    plan = rq.Plan(D, r, fx.U.astype(np.float32), fx.V.astype(np.float32))
+
+    sets = []
+    for i in range(NSETS):
+        kw = dict(n_outlier=w.n_outlier, outlier_scale=w.outlier_scale,
+                  dist=w.dist, seed=1000 * rank + i)
+        x = W.activations_bf16_fast(N, D, tensor_id=W.TID_X, device=str(dev), **kw)
+        res = W.activations_bf16_fast(N, D, tensor_id=W.TID_RESIDUAL,
+                                      device=str(dev), **kw)
+        if i == 0 and rank == 0:
+            x.copy_(fx.x.to(dev))
+            res.copy_(fx.residual.to(dev))
+        qw = torch.from_numpy(W.int4_packed_random(O_, K, i, W.TID_WEIGHTS)).to(dev)
+        sw = torch.from_numpy(W.weight_scales(O_, K, i)).to(dev)
+        sets.append((x, res, qw, sw))
+    h = torch.empty(N, D, dtype=torch.bfloat16, device=dev)
+    q = torch.empty(N, D // 2, dtype=torch.uint8, device=dev)
+    sc = torch.empty(N, dtype=torch.float32, device=dev)
+    out = torch.empty(N, O_, dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    sptr = stream.cuda_stream
+
+    def step(i):
+        x, res, qw, sw = sets[i % NSETS]
+        rq.respin_boundary_forward(plan, x, res, h, q, sc, sptr)
+        rq.w4a4_gemm(q, sc, qw, sw, out, sptr)
+
+    for i in range(max(3, args.warmup)):
+        step(i)
+    torch.cuda.synchronize()
+    if rq.respin_device_status() != 0:
+        raise RuntimeError("a kernel reported a device-side failure in warm-up")
+
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    time.sleep(0.05)
+
+    Ksteps = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)]
+          for _ in range(Ksteps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    wall0 = time.time()
+    t_start.record(stream)
+    for i in range(Ksteps):
+        x, res, qw, sw = sets[i % NSETS]
+        ev[i][0].record(stream)
+        rq.respin_boundary_forward(plan, x, res, h, q, sc, sptr)
+        ev[i][1].record(stream)
+        rq.w4a4_gemm(q, sc, qw, sw, out, sptr)
+        ev[i][2].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    wall1 = time.time()
+    if dist:
+        dist.barrier()
+    total_ms = t_start.elapsed_time(t_end)
+    b_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / Ksteps
+    g_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / Ksteps
+    clocks = sampler.summary(wall0, wall1)
+    if rq.respin_device_status() != 0:
+        raise RuntimeError("a kernel reported a device-side failure")
+
+    # ---- end to end through the public API with pinned host buffers
+    x_h = fx.x.pin_memory() if rank == 0 else sets[0][0].cpu().pin_memory()
+    r_h = fx.residual.pin_memory() if rank == 0 else sets[0][1].cpu().pin_memory()
+    x_d = torch.empty_like(sets[0][0])
+    r_d = torch.empty_like(sets[0][1])
+    out_h = torch.empty(N, O_, dtype=torch.bfloat16).pin_memory()
+    h_h = torch.empty(N, D, dtype=torch.bfloat16).pin_memory()
+    Ke = max(3, min(Ksteps, 50))
+
+    def e2e_step(i):
+        _, _, qw, sw = sets[i % NSETS]
+        x_d.copy_(x_h, non_blocking=True)
+        r_d.copy_(r_h, non_blocking=True)
+        rq.respin_boundary_forward(plan, x_d, r_d, h, q, sc, sptr)
+        rq.w4a4_gemm(q, sc, qw, sw, out, sptr)
+        out_h.copy_(out, non_blocking=True)
+        h_h.copy_(h, non_blocking=True)
+
+    for i in range(3):
+        e2e_step(i)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for i in range(Ke):
+        e2e_step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    e2e_ms = e0.elapsed_time(e1) / Ke
+    sampler.stop_evt.set()
+
+    times = torch.tensor([total_ms, e2e_ms, b_ms, g_ms], dtype=torch.float64,
+                         device=dev)
+    if dist:
+        dist.all_reduce(times, op=dist.ReduceOp.MAX)
+    total_ms, e2e_ms, b_ms, g_ms = times.tolist()
+    ms_step = total_ms / Ksteps
+
+    if rank == 0:
+        hbm_gbs, bf16_tf, src = peaks()
+        int8_tops = bf16_tf * INT8_OVER_BF16
+        gemm_ops = 2.0 * N * K * O_
+        gemm_tops = gemm_ops / (g_ms * 1e-3) / 1e12
+        b_bytes = N * (6.5 * D + 4) + 2 * D * 32 * 2
+        b_gbs = b_bytes / (b_ms * 1e-3) / 1e9
+        line = {
+            "metric": METRIC,
+            "value": world * N / (ms_step * 1e-3),
+            "unit": "tokens/s",
+            "n_gpus": world, "steps": Ksteps, "warmup": args.warmup,
+            "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16+int4", "data": "synthetic",
+            "config": config_block(w, world),
+            "boundary_tokens_per_s": world * N / (b_ms * 1e-3),
+            "boundary_us": b_ms * 1e3,
+            "gemm_tops": gemm_tops * world,
+            "gemm_us": g_ms * 1e3,
+            "roofline": {
+                "kernel": "w4a4_gemm_kernel", "bound": "tensor",
+                "achieved": gemm_tops, "peak": int8_tops, "unit": "TFLOP/s",
+                "frac": gemm_tops / int8_tops,
+                "traffic": traffic_for("w4a4_gemm_kernels.cuh", "w4a4_gemm_kernel"),
+                "peak_source": "%s bf16 burst %.1f TFLOP/s x %.0f (nominal "
+                               "int8/bf16 dense ratio); integer ops counted "
+                               "as 2 per multiply-add" % (src, bf16_tf,
+                                                          INT8_OVER_BF16)},
+            "roofline_boundary": {
+                "kernel": "boundary_cluster_kernel", "bound": "hbm",
+                "achieved": b_gbs, "peak": hbm_gbs, "unit": "GB/s",
+                "frac": b_gbs / hbm_gbs,
+                "traffic": traffic_for("boundary_kernels.cuh",
+                                       "boundary_cluster_kernel"),
+                "peak_source": "%s HBM copy bandwidth" % src},
+            "e2e": {"value": world * N / (e2e_ms * 1e-3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": 2 * N * D * 2,
+                    "d2h_bytes_per_step": N * O_ * 2 + N * D * 2},
+            "gpu_launches": 2 * Ksteps,
+            "clocks": clocks,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline_block(fx, qw_np, sw_np)
+        print(json.dumps(line), flush=True)
+    plan.destroy()
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_profile_launch(args):
+    """Warm-up launches, then exactly one more launch of the chosen kernel."""
+    import numpy as np
+    import torch
+    import rotation_post_quantization_b200 as rq
+    import workloads as W
+
+    w = W.WORKLOADS[WORKLOAD]
+    N = args.tokens or w.N
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    fx = W.workload_fixture(WORKLOAD, N=16)
+    plan = rq.Plan(w.D, w.r, fx.U.astype(np.float32), fx.V.astype(np.float32))
+    kw = dict(n_outlier=w.n_outlier, outlier_scale=w.outlier_scale, dist=w.dist)
+    x = W.activations_bf16_fast(N, w.D, tensor_id=W.TID_X, device="cuda", **kw)
+    res = W.activations_bf16_fast(N, w.D, tensor_id=W.TID_RESIDUAL, device="cuda", **kw)
+    h = torch.empty(N, w.D, dtype=torch.bfloat16, device=dev)
+    q = torch.empty(N, w.D // 2, dtype=torch.uint8, device=dev)
+    sc = torch.empty(N, dtype=torch.float32, device=dev)
+    qw = torch.from_numpy(W.int4_packed_random(w.O, w.D, 0, W.TID_WEIGHTS)).to(dev)
+    sw = torch.from_numpy(W.weight_scales(w.O, w.D, 0)).to(dev)
+    out = torch.empty(N, w.O, dtype=torch.bfloat16, device=dev)
+    rq.respin_boundary_forward(plan, x, res, h, q, sc)
+    for _ in range(args.warmup + 1):
+        if args.profile_launch == "boundary":
+            rq.respin_boundary_forward(plan, x, res, h, q, sc)
+        else:
+            rq.w4a4_gemm(q, sc, qw, sw, out)
+    torch.cuda.synchronize()
+    assert rq.respin_device_status() == 0
+    plan.destroy()
+    print("profile launch done: %s, %d tokens" % (args.profile_launch, N))
+
+
+def main():
+    args = parse_args()
+    if args.profile_launch:
+        run_profile_launch(args)
+        return
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+    run_ours(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    main()

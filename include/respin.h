@@ -1,0 +1,167 @@
+/*
+ * respin.h -- C ABI of the ReSpinQuant block-boundary library (B200, sm_100a).
+ *
+ * The library implements the inference-time hot path of "ReSpinQuant:
+ * Efficient Layer-Wise LLM Quantization via Subspace Residual Rotation
+ * Approximation" (arXiv 2604.11080, as explained on the gist.science pages in
+ * zh, it, nl, es and fr; cited below by language and section):
+ *
+ *   1. the per-token basis fix at a block boundary,
+ *        h' = residual * (I + U_r V_r^T) + x,
+ *      the rank-r form of the residual-path transition T = R_out^T R_in
+ *      (zh §2.1-§2.2; nl §2B-§2C; fr §2B-§2C), fused with
+ *   2. per-token symmetric INT4 quantization of h' (W4A4, zh §3-§4), and
+ *   3. the W4A4 GEMM that consumes those codes (zh §2.2: the linears stay
+ *      ordinary linears once the rotations are fused into their weights).
+ *
+ * Conventions for every call:
+ *   - Tokens are rows; tensors are row-major and contiguous.
+ *   - bf16 means IEEE bfloat16 (raw 16-bit storage), fp32 means IEEE binary32.
+ *   - INT4 codes are packed two per byte: element 2j in the low nibble of byte
+ *     j, element 2j+1 in the high nibble, two's complement (value & 0xF).
+ *   - All tensor pointers are DEVICE pointers owned by the caller, on the
+ *     device that is current when the call is made, 16-byte aligned unless
+ *     stated otherwise. The library never allocates per call.
+ *   - `stream` is a cudaStream_t handle (NULL = legacy default stream). Calls
+ *     are asynchronous: they validate, enqueue one kernel and return.
+ *   - Every call returns a respin_status_t. Validation errors are returned
+ *     before anything is enqueued; respin_last_error() then holds a message.
+ *     Kernels never trap: a kernel that gives up on a bounded wait records a
+ *     code in a device status word that respin_device_status() reads.
+ *   - No call is thread-safe with respect to the same plan being destroyed.
+ */
+#ifndef RESPIN_H_
+#define RESPIN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  RESPIN_OK = 0,
+  RESPIN_ERR_INVALID_ARG = 1,   /* null/negative/unknown argument          */
+  RESPIN_ERR_ALIGNMENT = 2,     /* a pointer is not suitably aligned        */
+  RESPIN_ERR_UNSUPPORTED = 3,   /* a size outside what the kernels support  */
+  RESPIN_ERR_CUDA = 4,          /* a CUDA runtime call failed               */
+  RESPIN_ERR_OOM = 5,           /* device allocation failed (plan creation) */
+  RESPIN_ERR_DEVICE_CHECK = 6   /* a kernel recorded a device-side failure  */
+} respin_status_t;
+
+typedef struct respin_plan_s* respin_plan_t;
+
+/* Plan flag: respin_boundary_forward writes h' as fp32 (the value before the
+ * bfloat16 rounding) instead of bf16. The codes are still computed from the
+ * bfloat16-rounded h'. Used to check the arithmetic of the fix directly. */
+#define RESPIN_H_FP32_DEBUG 1u
+
+/*
+ * respin_plan_create -- prepare the rank-r fix of one block boundary.
+ *
+ * Passage: the top-r SVD of Delta T = T - I gives the subspace in which the
+ * residual is rotated (it §2C; nl §2C; es §2B; fr §2C); with row vectors the
+ * fix is h (I + U_r V_r^T), which is the zh §2.2 form x + Q (M Q^T x) with
+ * U_r = Q and V_r = Q M.
+ *
+ *   out    : receives the plan handle.
+ *   D      : hidden size; D % 128 == 0, 128 <= D <= 65536.
+ *   r      : rank; 0 <= r <= 128 and r % 8 == 0. r == 0 gives plain
+ *            residual + x followed by quantization.
+ *   U_r    : HOST fp32 [D, r] row-major (may be NULL iff r == 0).
+ *   V_r    : HOST fp32 [D, r] row-major (may be NULL iff r == 0).
+ *   flags  : 0 or RESPIN_H_FP32_DEBUG.
+ *
+ * The plan rounds U_r and V_r to bfloat16 (round to nearest even), copies
+ * them to the current device (owned by the plan) and picks the launch
+ * configuration. Synchronous. Errors: INVALID_ARG, UNSUPPORTED (e.g. D*r too
+ * large for the on-chip factor slices), OOM, CUDA.
+ */
+respin_status_t respin_plan_create(respin_plan_t* out, int D, int r,
+                                   const float* U_r, const float* V_r,
+                                   unsigned flags);
+
+/* respin_plan_destroy -- free the plan's device factors. Waits for the device
+ * to finish outstanding work first. Unknown or already destroyed handles give
+ * INVALID_ARG. NULL is a no-op. */
+respin_status_t respin_plan_destroy(respin_plan_t plan);
+
+/*
+ * respin_boundary_forward -- fused block-boundary step for N tokens.
+ *
+ * Passage: the residual connection in the rotated basis needs the transition
+ * T before the addition (fr §2B; zh §2.2 "x_out = T x_in + ..."), applied in
+ * the rank-r subspace as projection, transform, re-projection and residual
+ * (zh §2.2 steps 1-3). Per token (row) n, in fp32 with the plan's bf16
+ * factors:
+ *     y      = residual[n] U_r                       (r values)
+ *     h[n]   = residual[n] + x[n] + y V_r^T
+ *     h'[n]  = bf16(h[n])                            (round to nearest even)
+ *     amax   = max_i |h'[n, i]|
+ *     inv    = 7 / amax, scale[n] = amax / 7         (binary32, RN)
+ *     q[n,i] = clamp(rint(h'[n,i] * inv), -8, 7)     (ties to even)
+ * A token with amax < 2^-125 gets scale 0 and all-zero codes.
+ *
+ *   plan      : from respin_plan_create; its device must be current.
+ *   x         : bf16 [N, D] block output (device).
+ *   residual  : bf16 [N, D] residual stream (device), or NULL for zero (then
+ *               h' = x and the factors are not used).
+ *   N         : tokens; N == 0 is a no-op; N < 0 is INVALID_ARG.
+ *   h_out     : bf16 [N, D] (fp32 [N, D] with RESPIN_H_FP32_DEBUG), or NULL
+ *               to skip writing h'.
+ *   q_packed  : uint8 [N, D/2] packed codes (device).
+ *   scale     : fp32 [N] per-token scales (device, 4-byte aligned).
+ *   stream    : cudaStream_t.
+ * No input may overlap an output. Errors: INVALID_ARG, ALIGNMENT, CUDA.
+ */
+respin_status_t respin_boundary_forward(respin_plan_t plan, const void* x,
+                                        const void* residual, int N,
+                                        void* h_out, uint8_t* q_packed,
+                                        float* scale, void* stream);
+
+/*
+ * w4a4_gemm -- out = bf16((float(acc) * scale_act[n]) * scale_w[o]) with
+ * acc[n, o] = sum_k a[n, k] w[o, k] exactly in int32 (W4A4 linear, zh §3-§4,
+ * fr §4; the weights already carry the fused rotations, zh §2.2).
+ *
+ *   q_act     : uint8 [N, K/2] packed activation codes (device).
+ *   scale_act : fp32 [N] per-token scales (device, 4-byte aligned).
+ *   q_w       : uint8 [O, K/2] packed weight codes, one row per output
+ *               channel (device).
+ *   scale_w   : fp32 [O] per-channel scales (device, 4-byte aligned).
+ *   N         : tokens (N == 0 is a no-op).
+ *   K         : reduction size; K % 128 == 0, 128 <= K <= 65536.
+ *   O         : output channels; O % 16 == 0, O >= 16.
+ *   out       : bf16 [N, O] (device).
+ * Both products of the epilogue round to nearest even in binary32; the
+ * integer sum is exact. Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, CUDA.
+ */
+respin_status_t w4a4_gemm(const uint8_t* q_act, const float* scale_act,
+                          const uint8_t* q_w, const float* scale_w, int N,
+                          int K, int O, void* out, void* stream);
+
+/* w4a4_gemm_i32 -- same contraction, writes the exact int32 accumulators
+ * acc_out [N, O] (device) instead of the scaled bf16 output. For tests. */
+respin_status_t w4a4_gemm_i32(const uint8_t* q_act, const uint8_t* q_w,
+                              int N, int K, int O, int32_t* acc_out,
+                              void* stream);
+
+/* respin_device_status -- synchronizes the current device, then returns and
+ * clears the device status word through *code (0 = no kernel gave up; else
+ * the site that gave up). Returns DEVICE_CHECK if *code != 0. */
+respin_status_t respin_device_status(int* code);
+
+/* respin_last_error -- message of the last failed call on this thread (empty
+ * string if none). The pointer stays valid until the next call on this
+ * thread. */
+const char* respin_last_error(void);
+
+/* respin_version -- library version string. */
+const char* respin_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RESPIN_H_ */

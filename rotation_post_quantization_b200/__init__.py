@@ -1,0 +1,168 @@
+"""Python binding of the ReSpinQuant block-boundary library (librespin.so).
+
+Argument marshalling only: every step of the path runs in the CUDA kernels
+behind the C ABI declared in include/respin.h. torch tensors supply device
+memory and the current CUDA stream. There is no CPU fallback: if the built
+library is missing, importing this package raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "librespin.so")
+
+RESPIN_OK = 0
+RESPIN_ERR_INVALID_ARG = 1
+RESPIN_ERR_ALIGNMENT = 2
+RESPIN_ERR_UNSUPPORTED = 3
+RESPIN_ERR_CUDA = 4
+RESPIN_ERR_OOM = 5
+RESPIN_ERR_DEVICE_CHECK = 6
+RESPIN_H_FP32_DEBUG = 1
+
+# Every entry point include/respin.h declares (checked by the tests).
+EXPORTED = ("respin_plan_create", "respin_plan_destroy",
+            "respin_boundary_forward", "w4a4_gemm", "w4a4_gemm_i32",
+            "respin_device_status", "respin_last_error", "respin_version")
+
+
+class RespinError(RuntimeError):
+    """A library call returned a status other than RESPIN_OK."""
+
+    def __init__(self, status: int, message: str):
+        super().__init__(f"respin status {status}: {message}")
+        self.status = status
+        self.message = message
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with "
+            "`python -m rotation_post_quantization_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i32, u32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_uint
+    fp = ctypes.POINTER(ctypes.c_float)
+    lib.respin_plan_create.argtypes = [ctypes.POINTER(vp), i32, i32, fp, fp, u32]
+    lib.respin_plan_destroy.argtypes = [vp]
+    lib.respin_boundary_forward.argtypes = [vp, vp, vp, i32, vp, vp, vp, vp]
+    lib.w4a4_gemm.argtypes = [vp, vp, vp, vp, i32, i32, i32, vp, vp]
+    lib.w4a4_gemm_i32.argtypes = [vp, vp, i32, i32, i32, vp, vp]
+    lib.respin_device_status.argtypes = [ctypes.POINTER(ctypes.c_int)]
+    for name in EXPORTED[:-2]:
+        getattr(lib, name).restype = ctypes.c_int
+    lib.respin_last_error.restype = ctypes.c_char_p
+    lib.respin_last_error.argtypes = []
+    lib.respin_version.restype = ctypes.c_char_p
+    lib.respin_version.argtypes = []
+    return lib
+
+
+lib = _load()
+
+
+def _check(status: int) -> None:
+    if status != RESPIN_OK:
+        raise RespinError(status, lib.respin_last_error().decode())
+
+
+def last_error() -> str:
+    return lib.respin_last_error().decode()
+
+
+def version() -> str:
+    return lib.respin_version().decode()
+
+
+def _ptr(t):
+    """Device pointer of a tensor (or None), as an int for ctypes."""
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream=None):
+    if stream is not None:
+        return stream if isinstance(stream, int) else stream.cuda_stream
+    import torch
+    return torch.cuda.current_stream().cuda_stream
+
+
+class Plan:
+    """respin_plan_create / respin_plan_destroy: one block boundary's factors."""
+
+    def __init__(self, D: int, r: int, U_r=None, V_r=None, flags: int = 0):
+        self.D, self.r, self.flags = int(D), int(r), int(flags)
+        self.handle = ctypes.c_void_p()
+        fp = ctypes.POINTER(ctypes.c_float)
+        U = V = None
+        if U_r is not None:
+            U = np.ascontiguousarray(U_r, dtype=np.float32)
+            V = np.ascontiguousarray(V_r, dtype=np.float32)
+            if U.shape != (self.D, self.r) or V.shape != (self.D, self.r):
+                raise ValueError("U_r and V_r must be [D, r]")
+        up = U.ctypes.data_as(fp) if U is not None else None
+        vp_ = V.ctypes.data_as(fp) if V is not None else None
+        _check(lib.respin_plan_create(ctypes.byref(self.handle), self.D,
+                                      self.r, up, vp_, self.flags))
+
+    def destroy(self) -> None:
+        if self.handle:
+            h, self.handle = self.handle, ctypes.c_void_p()
+            _check(lib.respin_plan_destroy(h))
+
+    def __del__(self):
+        try:
+            self.destroy()
+        except Exception:
+            pass
+
+
+def respin_plan_create(D, r, U_r=None, V_r=None, flags=0) -> Plan:
+    return Plan(D, r, U_r, V_r, flags)
+
+
+def respin_plan_destroy(plan: Plan) -> None:
+    plan.destroy()
+
+
+def respin_boundary_forward(plan: Plan, x, residual, h_out, q_packed, scale,
+                            stream=None) -> None:
+    """h' = residual (I + U_r V_r^T) + x, then per-token INT4 codes and scales.
+
+    x, residual, h_out: [N, D] CUDA tensors (bf16; h_out fp32 for a plan made
+    with RESPIN_H_FP32_DEBUG; residual / h_out may be None); q_packed: uint8
+    [N, D/2]; scale: fp32 [N].
+    """
+    N = int(x.shape[0]) if x is not None else 0
+    _check(lib.respin_boundary_forward(
+        plan.handle, _ptr(x), _ptr(residual), N, _ptr(h_out), _ptr(q_packed),
+        _ptr(scale), _stream(stream)))
+
+
+def w4a4_gemm(q_act, scale_act, q_w, scale_w, out, stream=None) -> None:
+    """out[N, O] (bf16) = (acc * scale_act[n]) * scale_w[o], acc exact int."""
+    N, K2 = q_act.shape
+    O = q_w.shape[0]
+    _check(lib.w4a4_gemm(_ptr(q_act), _ptr(scale_act), _ptr(q_w),
+                         _ptr(scale_w), int(N), int(2 * K2), int(O), _ptr(out),
+                         _stream(stream)))
+
+
+def w4a4_gemm_i32(q_act, q_w, acc_out, stream=None) -> None:
+    """acc_out[N, O] (int32) = exact integer dot products of the codes."""
+    N, K2 = q_act.shape
+    O = q_w.shape[0]
+    _check(lib.w4a4_gemm_i32(_ptr(q_act), _ptr(q_w), int(N), int(2 * K2),
+                             int(O), _ptr(acc_out), _stream(stream)))
+
+
+def respin_device_status() -> int:
+    """Synchronize and return (and clear) the device status word."""
+    code = ctypes.c_int(0)
+    st = lib.respin_device_status(ctypes.byref(code))
+    if st not in (RESPIN_OK, RESPIN_ERR_DEVICE_CHECK):
+        _check(st)
+    return code.value

@@ -1,0 +1,381 @@
+// Host side of the ReSpinQuant boundary library: the C ABI declared in
+// include/respin.h (argument validation, plans, launch configuration, error
+// reporting). One translation unit holds every kernel so that the device
+// status word is a single symbol without relocatable device code.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdint>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <set>
+#include <string>
+#include <vector>
+
+#include "respin.h"
+#include "ptx.cuh"
+#include "boundary_kernels.cuh"
+#include "w4a4_gemm_kernels.cuh"
+
+using namespace respin;
+
+namespace {
+
+thread_local std::string t_last_error;
+
+respin_status_t fail(respin_status_t st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  t_last_error = buf;
+  return st;
+}
+
+respin_status_t ok() {
+  return RESPIN_OK;
+}
+
+respin_status_t cuda_fail(cudaError_t e, const char* what) {
+  return fail(RESPIN_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+// Host-side fault hook: RESPIN_FAULT=<site> makes the named site fail as if
+// the underlying operation had failed, without touching the device. Sites:
+// "plan_alloc" (device allocation in plan creation) and "launch" (kernel
+// launch in the compute calls).
+bool fault_at(const char* site) {
+  const char* f = std::getenv("RESPIN_FAULT");
+  return f != nullptr && std::strcmp(f, site) == 0;
+}
+
+bool aligned(const void* p, size_t a) {
+  return (reinterpret_cast<uintptr_t>(p) % a) == 0;
+}
+
+// ------------------------------------------------------------ plans
+
+struct BoundaryConfig {
+  int T = 0, R = 0, cluster = 0, Dc = 0;
+  size_t smem = 0;
+  int max_clusters = 0;
+  const void* fn = nullptr;
+};
+
+}  // namespace
+
+struct respin_plan_s {
+  int D = 0, r = 0, r_pad = 0;
+  unsigned flags = 0;
+  int device = -1;
+  __nv_bfloat16* factors = nullptr;  // [r_pad, D] U^T then [D, r_pad] V
+  BoundaryConfig cfg;
+};
+
+namespace {
+
+std::mutex g_plans_mu;
+std::set<respin_plan_s*> g_plans;
+
+bool plan_alive(respin_plan_s* p) {
+  std::lock_guard<std::mutex> lk(g_plans_mu);
+  return g_plans.count(p) != 0;
+}
+
+template <int T, int R, bool F32>
+const void* cluster_fn() {
+  return reinterpret_cast<const void*>(&boundary_cluster_kernel<T, R, F32>);
+}
+
+const void* pick_cluster_fn(int T, int R, bool f32) {
+#define RESPIN_PICK(TT, RR)                                                   \
+  if (T == TT && R == RR) return f32 ? cluster_fn<TT, RR, true>() : cluster_fn<TT, RR, false>();
+  RESPIN_PICK(32, 16) RESPIN_PICK(32, 32) RESPIN_PICK(32, 64)
+  RESPIN_PICK(16, 16) RESPIN_PICK(16, 32) RESPIN_PICK(16, 64) RESPIN_PICK(16, 128)
+#undef RESPIN_PICK
+  return nullptr;
+}
+
+// Choose cluster size and token tile: the smallest cluster whose per-CTA
+// slice (resident U^T and V slices plus a two-stage residual/x ring) fits in
+// shared memory, preferring 32-token tiles.
+respin_status_t configure_boundary(int D, int R, bool f32, BoundaryConfig* out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  int smem_optin = 0;
+  e = cudaDeviceGetAttribute(&smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+  const int clusters[] = {1, 2, 4, 8, 16};
+  const int tiles[] = {32, 16};
+  for (int C : clusters) {
+    if (D % C) continue;
+    const int Dc = D / C;
+    if (Dc % 64) continue;
+    for (int T : tiles) {
+      if (T * R > 2048) continue;
+      const void* fn = pick_cluster_fn(T, R, f32);
+      if (!fn) continue;
+      const size_t smem = boundary_smem_layout(T, R, Dc).total;
+      if (smem > static_cast<size_t>(smem_optin)) continue;
+      e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(smem)");
+      if (C > 8) {
+        e = cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        if (e != cudaSuccess) { cudaGetLastError(); continue; }
+      }
+      cudaLaunchConfig_t lc = {};
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = C;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      lc.gridDim = dim3(C, 1, 1);
+      lc.blockDim = dim3(kBoundaryThreads, 1, 1);
+      lc.dynamicSmemBytes = smem;
+      lc.attrs = attr;
+      lc.numAttrs = 1;
+      int nclusters = 0;
+      e = cudaOccupancyMaxActiveClusters(&nclusters, fn, &lc);
+      if (e != cudaSuccess || nclusters <= 0) { cudaGetLastError(); continue; }
+      out->T = T; out->R = R; out->cluster = C; out->Dc = Dc;
+      out->smem = smem; out->max_clusters = nclusters; out->fn = fn;
+      return ok();
+    }
+  }
+  return fail(RESPIN_ERR_UNSUPPORTED,
+              "no cluster configuration holds the factor slices for D=%d, padded r=%d", D, R);
+}
+
+respin_status_t check_device(int want) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev != want)
+    return fail(RESPIN_ERR_INVALID_ARG, "plan was created on device %d but device %d is current",
+                want, dev);
+  return ok();
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* respin_last_error(void) { return t_last_error.c_str(); }
+
+const char* respin_version(void) { return "respin-b200 0.1 (sm_100a)"; }
+
+respin_status_t respin_plan_create(respin_plan_t* out, int D, int r, const float* U_r,
+                                   const float* V_r, unsigned flags) {
+  t_last_error.clear();
+  if (out == nullptr) return fail(RESPIN_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  if (D < 128 || D > 65536 || D % 128)
+    return fail(RESPIN_ERR_UNSUPPORTED, "D=%d: need 128 <= D <= 65536 and D %% 128 == 0", D);
+  if (r < 0 || r > 128 || r % 8)
+    return fail(RESPIN_ERR_UNSUPPORTED, "r=%d: need 0 <= r <= 128 and r %% 8 == 0", r);
+  if (r > 0 && (U_r == nullptr || V_r == nullptr))
+    return fail(RESPIN_ERR_INVALID_ARG, "U_r and V_r must be non-NULL when r > 0");
+  if (flags & ~RESPIN_H_FP32_DEBUG) return fail(RESPIN_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
+  const int r_pad = r == 0 ? 0 : (r <= 16 ? 16 : r <= 32 ? 32 : r <= 64 ? 64 : 128);
+  if (fault_at("plan_alloc")) return fail(RESPIN_ERR_OOM, "injected fault at plan_alloc");
+
+  respin_plan_s* p = new respin_plan_s();
+  p->D = D; p->r = r; p->r_pad = r_pad; p->flags = flags;
+  cudaError_t e = cudaGetDevice(&p->device);
+  if (e != cudaSuccess) { delete p; return cuda_fail(e, "cudaGetDevice"); }
+  if (r > 0) {
+    respin_status_t st = configure_boundary(D, r_pad, (flags & RESPIN_H_FP32_DEBUG) != 0, &p->cfg);
+    if (st != RESPIN_OK) { delete p; return st; }
+    // Factors as bf16 (round to nearest even): U^T [r_pad, D] then V [D, r_pad].
+    std::vector<__nv_bfloat16> host(static_cast<size_t>(2) * r_pad * D, __float2bfloat16_rn(0.f));
+    __nv_bfloat16* ut = host.data();
+    __nv_bfloat16* v = host.data() + static_cast<size_t>(r_pad) * D;
+    for (int d = 0; d < D; ++d)
+      for (int j = 0; j < r; ++j) {
+        ut[static_cast<size_t>(j) * D + d] = __float2bfloat16_rn(U_r[static_cast<size_t>(d) * r + j]);
+        v[static_cast<size_t>(d) * r_pad + j] = __float2bfloat16_rn(V_r[static_cast<size_t>(d) * r + j]);
+      }
+    e = cudaMalloc(&p->factors, host.size() * sizeof(__nv_bfloat16));
+    if (e != cudaSuccess) { delete p; cudaGetLastError(); return fail(RESPIN_ERR_OOM, "cudaMalloc factors: %s", cudaGetErrorString(e)); }
+    e = cudaMemcpy(p->factors, host.data(), host.size() * sizeof(__nv_bfloat16), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) { cudaFree(p->factors); delete p; return cuda_fail(e, "cudaMemcpy factors"); }
+  }
+  // The row kernels need the shared-memory carve-out only for their reduction.
+  {
+    std::lock_guard<std::mutex> lk(g_plans_mu);
+    g_plans.insert(p);
+  }
+  *out = p;
+  return ok();
+}
+
+respin_status_t respin_plan_destroy(respin_plan_t plan) {
+  t_last_error.clear();
+  if (plan == nullptr) return ok();
+  {
+    std::lock_guard<std::mutex> lk(g_plans_mu);
+    if (!g_plans.erase(plan)) return fail(RESPIN_ERR_INVALID_ARG, "unknown or destroyed plan");
+  }
+  respin_status_t st = RESPIN_OK;
+  if (plan->factors) {
+    int cur = -1;
+    cudaGetDevice(&cur);
+    cudaSetDevice(plan->device);
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e == cudaSuccess) e = cudaFree(plan->factors);
+    if (e != cudaSuccess) st = cuda_fail(e, "releasing plan factors");
+    cudaSetDevice(cur);
+  }
+  delete plan;
+  return st;
+}
+
+respin_status_t respin_boundary_forward(respin_plan_t plan, const void* x, const void* residual,
+                                        int N, void* h_out, uint8_t* q_packed, float* scale,
+                                        void* stream) {
+  t_last_error.clear();
+  if (plan == nullptr || !plan_alive(plan)) return fail(RESPIN_ERR_INVALID_ARG, "unknown or destroyed plan");
+  if (N < 0) return fail(RESPIN_ERR_INVALID_ARG, "N=%d is negative", N);
+  if (N == 0) return ok();
+  if (x == nullptr || q_packed == nullptr || scale == nullptr)
+    return fail(RESPIN_ERR_INVALID_ARG, "x, q_packed and scale must be non-NULL");
+  if (!aligned(x, 16) || !aligned(residual, 16) || !aligned(h_out, 16) || !aligned(q_packed, 16))
+    return fail(RESPIN_ERR_ALIGNMENT, "x, residual, h_out and q_packed must be 16-byte aligned");
+  if (!aligned(scale, 4)) return fail(RESPIN_ERR_ALIGNMENT, "scale must be 4-byte aligned");
+  if (fault_at("launch")) return fail(RESPIN_ERR_CUDA, "injected fault at launch");
+  respin_status_t st = check_device(plan->device);
+  if (st != RESPIN_OK) return st;
+
+  const int D = plan->D;
+  const bool f32 = (plan->flags & RESPIN_H_FP32_DEBUG) != 0;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bf16* xb = static_cast<const bf16*>(x);
+  const bf16* rb = static_cast<const bf16*>(residual);
+
+  if (plan->r == 0 || residual == nullptr) {
+    int sms = 148;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, plan->device);
+    const int grid = N < sms * 16 ? N : sms * 16;
+    if (D <= 256 * 64) {
+      if (f32) boundary_rowwise_kernel<256, true><<<grid, 256, 0, s>>>(xb, rb, N, D, h_out, q_packed, scale);
+      else boundary_rowwise_kernel<256, false><<<grid, 256, 0, s>>>(xb, rb, N, D, h_out, q_packed, scale);
+    } else {
+      if (f32) boundary_rowwise_kernel<1024, true><<<grid, 1024, 0, s>>>(xb, rb, N, D, h_out, q_packed, scale);
+      else boundary_rowwise_kernel<1024, false><<<grid, 1024, 0, s>>>(xb, rb, N, D, h_out, q_packed, scale);
+    }
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "boundary_rowwise_kernel launch");
+    return ok();
+  }
+
+  const BoundaryConfig& c = plan->cfg;
+  const int ntiles = (N + c.T - 1) / c.T;
+  const int nclusters = ntiles < c.max_clusters ? ntiles : c.max_clusters;
+  cudaLaunchConfig_t lc = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = c.cluster;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  lc.gridDim = dim3(nclusters * c.cluster, 1, 1);
+  lc.blockDim = dim3(kBoundaryThreads, 1, 1);
+  lc.dynamicSmemBytes = c.smem;
+  lc.stream = s;
+  lc.attrs = attr;
+  lc.numAttrs = 1;
+  const bf16* ut = plan->factors;
+  const bf16* v = plan->factors + static_cast<size_t>(plan->r_pad) * D;
+  int Dc = c.Dc;
+  void* args[] = {&xb, &rb, &ut, &v, &N, const_cast<int*>(&D), &Dc, &h_out, &q_packed, &scale};
+  cudaError_t e = cudaLaunchKernelExC(&lc, c.fn, args);
+  if (e != cudaSuccess) return cuda_fail(e, "boundary_cluster_kernel launch");
+  return ok();
+}
+
+// The GEMM kernels need the large dynamic shared-memory carve-out; set it
+// once per device.
+static cudaError_t gemm_prepare(int dev) {
+  static std::mutex mu;
+  static bool done[256] = {};
+  if (dev < 0 || dev >= 256) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lk(mu);
+  if (done[dev]) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(&w4a4_gemm_kernel<false>),
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmemBytes);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(reinterpret_cast<const void*>(&w4a4_gemm_kernel<true>),
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmemBytes);
+  if (e == cudaSuccess) done[dev] = true;
+  return e;
+}
+
+static respin_status_t gemm_common(const uint8_t* q_act, const float* scale_act, const uint8_t* q_w,
+                                   const float* scale_w, int N, int K, int O, void* out,
+                                   void* stream, bool i32) {
+  t_last_error.clear();
+  if (N < 0) return fail(RESPIN_ERR_INVALID_ARG, "N=%d is negative", N);
+  if (K < 128 || K > 65536 || K % 128)
+    return fail(RESPIN_ERR_UNSUPPORTED, "K=%d: need 128 <= K <= 65536 and K %% 128 == 0", K);
+  if (O < 16 || O % 16) return fail(RESPIN_ERR_UNSUPPORTED, "O=%d: need O >= 16 and O %% 16 == 0", O);
+  if (N == 0) return ok();
+  if (q_act == nullptr || q_w == nullptr || out == nullptr || (!i32 && (scale_act == nullptr || scale_w == nullptr)))
+    return fail(RESPIN_ERR_INVALID_ARG, "a required pointer is NULL");
+  if (!aligned(q_act, 16) || !aligned(q_w, 16) || !aligned(out, 16))
+    return fail(RESPIN_ERR_ALIGNMENT, "q_act, q_w and out must be 16-byte aligned");
+  if (!aligned(scale_act, 4) || !aligned(scale_w, 4))
+    return fail(RESPIN_ERR_ALIGNMENT, "scales must be 4-byte aligned");
+  if (static_cast<long long>((N + kGemmBM - 1) / kGemmBM) > 65535)
+    return fail(RESPIN_ERR_UNSUPPORTED, "N=%d too large", N);
+  if (fault_at("launch")) return fail(RESPIN_ERR_CUDA, "injected fault at launch");
+
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  e = gemm_prepare(dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gemm smem)");
+  dim3 grid((O + kGemmBN - 1) / kGemmBN, (N + kGemmBM - 1) / kGemmBM, 1);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (i32)
+    w4a4_gemm_kernel<true><<<grid, kGemmThreads, kGemmSmemBytes, s>>>(q_act, scale_act, q_w, scale_w, N, K, O, out);
+  else
+    w4a4_gemm_kernel<false><<<grid, kGemmThreads, kGemmSmemBytes, s>>>(q_act, scale_act, q_w, scale_w, N, K, O, out);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "w4a4_gemm_kernel launch");
+  return ok();
+}
+
+respin_status_t w4a4_gemm(const uint8_t* q_act, const float* scale_act, const uint8_t* q_w,
+                          const float* scale_w, int N, int K, int O, void* out, void* stream) {
+  return gemm_common(q_act, scale_act, q_w, scale_w, N, K, O, out, stream, false);
+}
+
+respin_status_t w4a4_gemm_i32(const uint8_t* q_act, const uint8_t* q_w, int N, int K, int O,
+                              int32_t* acc_out, void* stream) {
+  return gemm_common(q_act, nullptr, q_w, nullptr, N, K, O, acc_out, stream, true);
+}
+
+respin_status_t respin_device_status(int* code) {
+  t_last_error.clear();
+  if (code == nullptr) return fail(RESPIN_ERR_INVALID_ARG, "code is NULL");
+  *code = 0;
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+  int v = 0;
+  e = cudaMemcpyFromSymbol(&v, g_status, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e, "reading the device status word");
+  if (v != 0) {
+    const int zero = 0;
+    e = cudaMemcpyToSymbol(g_status, &zero, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the device status word");
+    *code = v;
+    return fail(RESPIN_ERR_DEVICE_CHECK, "a kernel gave up on a bounded wait (site %d)", v);
+  }
+  return ok();
+}
+
+}  // extern "C"
