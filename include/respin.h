@@ -129,7 +129,7 @@ respin_status_t respin_boundary_forward(respin_plan_t plan, const void* x,
  *   scale_act : fp32 [N] per-token scales (device, 4-byte aligned).
  *   q_w       : uint8 [O, K/2] packed weight codes, one row per output
  *               channel (device).
- *   scale_w   : fp32 [O] per-channel scales (device, 4-byte aligned).
+ *   scale_w   : fp32 [O] per-channel scales (device, 16-byte aligned).
  *   N         : tokens (N == 0 is a no-op).
  *   K         : reduction size; K % 128 == 0, 128 <= K <= 65536.
  *   O         : output channels; O % 16 == 0, O >= 16.

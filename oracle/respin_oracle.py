@@ -249,6 +249,20 @@ def w4a4_acc(q_act_packed, q_w_packed) -> np.ndarray:
     return a @ w.T
 
 
+def w4a4_acc_fp64(q_act_packed, q_w_packed) -> np.ndarray:
+    """The same integer sums through a float64 matrix product (fast).
+
+    Exact: every product is an integer of magnitude <= 64 and every partial
+    sum has magnitude <= 64 K < 2^53, so no float64 rounding occurs in any
+    summation order.
+    """
+    a = unpack_int4(q_act_packed).astype(np.float64)
+    w = unpack_int4(q_w_packed).astype(np.float64)
+    if 64 * a.shape[1] >= 2 ** 53:
+        raise ValueError("K too large for an exact float64 product")
+    return (a @ w.T).astype(np.int64)
+
+
 def w4a4_epilogue_bits(acc, scale_act, scale_w) -> np.ndarray:
     """bf16 bits of (float(acc) * sa[n]) * sw[o], binary32 throughout."""
     acc = np.asarray(acc, np.int64)

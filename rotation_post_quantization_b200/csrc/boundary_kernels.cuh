@@ -2,25 +2,35 @@
 //
 // Per token (row) n, with the plan's bfloat16 factors U (D x r) and V (D x r):
 //   y = residual[n] U ;  h = (residual[n] + x[n]) + y V^T  (fp32)
-//   h' = bf16(h) ; amax = max|h'| ; inv = 7/amax ; q = clamp(rint(h' inv), -8, 7)
+//   h' = bf16(h) ; amax = max|h'| ; inv = 7/amax ; q = rint(h' inv)
 // This is the subspace residual rotation of the ReSpinQuant explainers (zh page
 // §2.2 steps 1-3: projection, transform inside the subspace, re-projection and
 // residual) in the row convention, followed by 4-bit activation quantization
-// (zh §3-§4, W4A4).
+// (zh §3-§4, W4A4). Since |h'| <= amax, |fl(h' * fl(7/amax))| <= 7 (1+2^-24)^2
+// < 7.5, so the code is always in [-7, 7] and no clamp is needed.
 //
-// Cluster kernel design (B200): a token tile of T rows is split along D over a
-// thread-block cluster of C CTAs (one per SM). CTA c owns columns
-// [c*Dc, (c+1)*Dc) and keeps its slices of U^T and V resident in shared memory
-// for the whole (persistent) launch, so the factors are read from L2 once per
-// CTA, not once per tile. Residual and x tiles arrive by 1-D bulk copies into
-// a two-stage shared-memory ring (next tile in flight while this one is
-// computed). The two whole-row dependencies - y needs the full row before the
-// re-projection, amax needs the full row before quantization - are resolved
-// with two cluster barriers per tile and distributed-shared-memory reads. Both
-// skinny products run on tensor cores (mma.sync m16n8k16 bf16, fp32
-// accumulate); y is split into bf16 hi + lo parts for the second product so
-// that it keeps ~16 mantissa bits. HBM sees each input byte once and each
-// output byte once.
+// Cluster design (B200): a tile of T tokens is split along D over a
+// thread-block cluster of C CTAs (one per SM); CTA c owns the columns
+// [c*Dc, (c+1)*Dc) of every token in the tile and works through the tiles of
+// its cluster in a persistent loop. Residual and x tiles arrive by 1-D bulk
+// copies (one per row) into a shared-memory ring, so later tiles are in
+// flight while one is computed. The two whole-row dependencies - y needs the
+// full row before the re-projection, amax needs the full row before
+// quantization - are resolved with a cluster barrier each and
+// distributed-shared-memory reads (all remote loads of a value in flight at
+// once, summed in rank order so every CTA gets the identical y). Both skinny
+// products run on tensor cores (mma.sync m16n8k16 bf16, fp32 accumulate); y is
+// split into bf16 hi + lo parts for the re-projection, keeping ~16 mantissa
+// bits. HBM sees each input byte once and each output byte once.
+//
+// Two variants:
+//  * boundary_cluster_rf_kernel (r <= 32): each CTA keeps its slices of U and V
+//    in REGISTERS for the whole launch, loaded once from a fragment-ordered
+//    copy that the plan prepares (coalesced 16-byte loads), which leaves the
+//    shared memory to a 3-stage tile ring.
+//  * boundary_cluster_smem_kernel (r = 64, 128): the factor slices live in
+//    shared memory (U^T with padded rows, V with 16-byte chunks swizzled),
+//    2-stage tile ring.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -35,52 +45,6 @@ using bf16 = __nv_bfloat16;
 constexpr int kBoundaryThreads = 256;
 constexpr float kZeroTokenAmax = 2.3509887e-38f;  // 2^-125
 
-template <int T, int R>
-struct BoundaryCfg {
-  static constexpr int kWarps = kBoundaryThreads / 32;
-  static constexpr int MT = T / 16;                       // m16 tiles per token tile
-  static constexpr int NT1 = R / 8;                       // n8 tiles of y
-  static constexpr int WN = (NT1 / 4) > 1 ? NT1 / 4 : 1;  // warps along r (phase 1)
-  static constexpr int WK = kWarps / (MT * WN);           // warps along Dc (phase 1)
-  static constexpr int NPW = NT1 / WN;                    // n8 tiles per warp (2 or 4)
-  static constexpr int KS2 = R / 16;                      // k16 steps of phase 2
-  static constexpr int CPR = R / 8;                       // 16-byte chunks per V row
-  static constexpr int VL = (8 / CPR) > 1 ? 8 / CPR : 1;  // V rows per 128-byte line
-  static constexpr int VXM = (CPR < 8 ? CPR : 8) - 1;     // chunk swizzle mask
-  static_assert(T == 16 || T == 32, "token tile");
-  static_assert(R == 16 || R == 32 || R == 64 || R == 128, "padded rank");
-  static_assert(MT * WN * WK == kWarps, "warp split");
-  static_assert(NPW == 2 || NPW == 4, "phase-1 n tiles per warp");
-};
-
-// Shared-memory carve-up of the cluster kernel (identical on host and device).
-struct BoundarySmem {
-  uint32_t us, vs, stage[2][2], partial, ybuf, yfull, wamax, amaxbuf, rowinv, bars, total;
-};
-
-__host__ __device__ inline BoundarySmem boundary_smem_layout(int T, int R, int Dc) {
-  const int MT = T / 16, NT1 = R / 8;
-  const int WN = (NT1 / 4) > 1 ? NT1 / 4 : 1;
-  const int WK = 8 / (MT * WN);
-  const uint32_t pitch = static_cast<uint32_t>(Dc) * 2 + 16;
-  BoundarySmem L;
-  uint32_t off = 0;
-  L.us = off;       off += R * pitch;                       // U^T slice, padded rows
-  L.vs = off;       off += static_cast<uint32_t>(Dc) * R * 2;  // V slice, swizzled
-  for (int s = 0; s < 2; ++s)
-    for (int t = 0; t < 2; ++t) { L.stage[s][t] = off; off += T * pitch; }
-  L.partial = off;  off += WK * T * R * 4;
-  L.ybuf = off;     off += T * R * 4;
-  L.yfull = off;    off += T * R * 4;
-  L.wamax = off;    off += 8 * T * 4;
-  L.amaxbuf = off;  off += T * 4;
-  L.rowinv = off;   off += T * 4;
-  off = (off + 15u) & ~15u;
-  L.bars = off;     off += 4 * 8;
-  L.total = off;
-  return L;
-}
-
 __device__ __forceinline__ float bf16_lo_f32(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi_f32(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
@@ -92,8 +56,7 @@ __device__ __forceinline__ uint32_t quantize8(const uint4 hv, float inv) {
   for (int e = 0; e < 8; ++e) {
     const uint32_t word = w[e >> 1];
     const float f = (e & 1) ? bf16_hi_f32(word) : bf16_lo_f32(word);
-    int q = __float2int_rn(__fmul_rn(f, inv));
-    q = min(max(q, -8), 7);
+    const int q = __float2int_rn(__fmul_rn(f, inv));
     packed |= (static_cast<uint32_t>(q) & 0xFu) << (4 * e);
   }
   return packed;
@@ -109,14 +72,495 @@ __device__ __forceinline__ void inv_and_scale(float amax, float& inv, float& sca
   }
 }
 
+// y in fp32 (two floats) -> bf16x2 hi and lo parts with hi + lo ~ y.
+__device__ __forceinline__ void split_bf16x2(float2 v, uint32_t& hi, uint32_t& lo) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(v.x, v.y);
+  const float2 hf = __bfloat1622float2(h);
+  const __nv_bfloat162 l = __floats2bfloat162_rn(v.x - hf.x, v.y - hf.y);
+  hi = *reinterpret_cast<const uint32_t*>(&h);
+  lo = *reinterpret_cast<const uint32_t*>(&l);
+}
+
+// Stage the residual and x rows of one tile with 1-D bulk copies (warp 0;
+// lane i copies row i). Rows past N are not copied.
+__device__ __forceinline__ void stage_tile(const bf16* __restrict__ x, const bf16* __restrict__ res,
+                                           int row0, int N, int D, int col0, int Dc, int T,
+                                           uint32_t rdst, uint32_t xdst, uint32_t pitch,
+                                           uint32_t bar_r, uint32_t bar_x, int lane) {
+  const int rows = min(T, N - row0);
+  const uint32_t bytes = static_cast<uint32_t>(Dc) * 2;
+  if (lane == 0) {
+    mbar_arrive_expect_tx(bar_r, rows * bytes);
+    mbar_arrive_expect_tx(bar_x, rows * bytes);
+  }
+  __syncwarp();
+  if (lane < rows) {
+    const size_t gofs = static_cast<size_t>(row0 + lane) * D + col0;
+    bulk_g2s(rdst + lane * pitch, res + gofs, bytes, bar_r);
+    bulk_g2s(xdst + lane * pitch, x + gofs, bytes, bar_x);
+  }
+}
+
+// Epilogue of one n8 column block of the re-projection for the rows of one
+// m16 tile: h = (res + x) + corr, bf16 round in place (into the x slot),
+// row amax, optional fp32 store.
+template <bool F32OUT>
+__device__ __forceinline__ void finish_n8(const float (&acc)[4], const uint8_t* rs_ptr, uint8_t* xs_ptr,
+                                          uint32_t pitch, int rowA, int colc, float (&rmax)[2],
+                                          void* h_out, int row0, int N, int D, int col0) {
+#pragma unroll
+  for (int hh = 0; hh < 2; ++hh) {
+    const int row = rowA + 8 * hh;
+    const uint32_t off = row * pitch + colc * 2;
+    const uint32_t rw = *reinterpret_cast<const uint32_t*>(rs_ptr + off);
+    const uint32_t xw = *reinterpret_cast<const uint32_t*>(xs_ptr + off);
+    const float h0 = (bf16_lo_f32(rw) + bf16_lo_f32(xw)) + acc[2 * hh];
+    const float h1 = (bf16_hi_f32(rw) + bf16_hi_f32(xw)) + acc[2 * hh + 1];
+    const uint32_t hb = pack_bf16x2(h0, h1);
+    *reinterpret_cast<uint32_t*>(xs_ptr + off) = hb;
+    rmax[hh] = fmaxf(rmax[hh], fmaxf(fabsf(bf16_lo_f32(hb)), fabsf(bf16_hi_f32(hb))));
+    if constexpr (F32OUT) {
+      if (h_out != nullptr && row0 + row < N) {
+        float* hf = static_cast<float*>(h_out) + static_cast<size_t>(row0 + row) * D + col0 + colc;
+        *reinterpret_cast<float2*>(hf) = make_float2(h0, h1);
+      }
+    }
+  }
+}
+
+// Row amax: per-thread row maxima -> warp maxima in `wamax` [8][T] -> after a
+// CTA barrier the T row maxima of this CTA's slice in `amaxbuf`.
+template <int MT, int T>
+__device__ __forceinline__ void publish_amax(float (&rmax)[MT][2], float* wamax, float* amaxbuf,
+                                             int warp, int lane, int tid) {
+  const int g = lane >> 2, q4 = lane & 3;
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      float m = rmax[mt][hh];
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+      if (q4 == 0) wamax[warp * T + mt * 16 + g + 8 * hh] = m;
+    }
+  __syncthreads();
+  if (tid < T) {
+    float m = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) m = fmaxf(m, wamax[w * T + tid]);
+    amaxbuf[tid] = m;
+  }
+}
+
+// After the amax cluster barrier: gather every CTA's row maxima in parallel
+// (one remote load per thread), reduce, and set the rows' 1/scale factors.
+template <int T>
+__device__ __forceinline__ void gather_amax(uint32_t amaxbuf_addr, float* am2, float* rowinv,
+                                            float* scale_out, uint32_t csize, uint32_t crank,
+                                            int row0, int N, int tid) {
+  for (int i = tid; i < static_cast<int>(csize) * T; i += kBoundaryThreads) {
+    const uint32_t c = static_cast<uint32_t>(i / T);
+    am2[i] = ld_dsmem_f32(map_to_rank(amaxbuf_addr + 4u * (i % T), c));
+  }
+  __syncthreads();
+  if (tid < T) {
+    float m = 0.f;
+    for (uint32_t c = 0; c < csize; ++c) m = fmaxf(m, am2[c * T + tid]);
+    float inv, sc;
+    inv_and_scale(m, inv, sc);
+    rowinv[tid] = inv;
+    if (crank == 0 && row0 + tid < N) scale_out[row0 + tid] = sc;
+  }
+  __syncthreads();
+}
+
+// Store h' (bf16) and the packed codes of this CTA's slice of the tile.
+template <bool F32OUT>
+__device__ __forceinline__ void store_tile(const uint8_t* xs_ptr, uint32_t pitch, const float* rowinv,
+                                           int T, int Dc, int row0, int N, int D, int col0,
+                                           void* h_out, uint8_t* q_out, int tid) {
+  const int vpr = Dc / 8;
+  for (int i = tid; i < T * vpr; i += kBoundaryThreads) {
+    const int row = i / vpr, v = i % vpr;
+    if (row0 + row >= N) continue;
+    const uint4 hv = *reinterpret_cast<const uint4*>(xs_ptr + row * pitch + v * 16);
+    const size_t gi = static_cast<size_t>(row0 + row) * D + col0 + v * 8;
+    if constexpr (!F32OUT) {
+      if (h_out != nullptr) *reinterpret_cast<uint4*>(static_cast<bf16*>(h_out) + gi) = hv;
+    }
+    *reinterpret_cast<uint32_t*>(q_out + gi / 2) = quantize8(hv, rowinv[row]);
+  }
+}
+
+// ============================================================================
+// Register-resident factors (r <= 32): T tokens per tile, Dc columns per CTA,
+// 3-stage tile ring. Warp 0 stages the tile two ahead while it waits at the
+// tile's two cluster barriers (residual rows at the first, x rows at the
+// second), so the copy issue overlaps the barrier latency. 8 warps keep the
+// 255-register budget that the resident fragments need.
+// ============================================================================
+
+constexpr int kRfThreads = 256;
+
+template <int R, int T, int Dc>
+struct RfCfg {
+  static constexpr int S = 3;
+  static constexpr int MT = T / 16;            // m16 tiles per token tile
+  static constexpr int WK = 8 / MT;            // warps along Dc in phase 1
+  static constexpr int KS = Dc / 16;           // k16 steps of phase 1
+  static constexpr int KPW = KS / WK;          // k16 steps per warp in phase 1
+  static constexpr int NPW = R / 8;            // n8 tiles of y per warp (all of r)
+  static constexpr int KS2 = R / 16;           // k16 steps of the re-projection
+  static constexpr int NTW = Dc / 64;          // n8 column tiles per warp (phase 2)
+  static constexpr int UREG = KPW * NPW * 2;   // 32-bit U fragment registers per lane
+  static constexpr int VREG = NTW * KS2 * 2;   // 32-bit V fragment registers per lane
+  static constexpr int RP = R + 8;             // padded fp32 row (conflict-free float2)
+  static constexpr uint32_t pitch = Dc * 2 + 16;
+  static constexpr uint32_t kStage = 2 * T * pitch;           // residual rows, then x rows
+  static constexpr uint32_t oPart = S * kStage;               // [WK][T][RP]; y aliases [0]
+  static constexpr uint32_t oYbuf = oPart + WK * T * RP * 4;  // [T][R] this CTA's partial y
+  static constexpr uint32_t oWamax = oYbuf + T * R * 4;       // [8][T]
+  static constexpr uint32_t oAm2 = oWamax + 8 * T * 4;        // [16][T]
+  static constexpr uint32_t oAmax = oAm2 + 16 * T * 4;        // [T]
+  static constexpr uint32_t oRinv = oAmax + T * 4;            // [T]
+  static constexpr uint32_t oBars = oRinv + T * 4;            // full_res[S], full_x[S]
+  static constexpr uint32_t kSmem = oBars + 2 * S * 8;
+  static_assert(R == 16 || R == 32, "register-resident factors need r <= 32");
+  static_assert(T == 16 || T == 32, "token tile");
+  static_assert(KS % WK == 0 && Dc % 64 == 0, "column slice");
+  static_assert(UREG % 4 == 0 && VREG % 4 == 0, "fragment chunks");
+  static_assert(T * R / 4 <= kRfThreads, "one float4 of y per thread");
+};
+
+// 8 bf16 values -> 8 packed INT4 codes using round-to-nearest-even by
+// addition: for |t| < 2^22, fl(t + 1.5*2^23) = 1.5*2^23 + rint(t) (ties to
+// even), and its low 4 bits are rint(t) mod 16, the two's-complement nibble.
+// t = fl(g * inv) exactly as in the definition (separate multiply and add).
+__device__ __forceinline__ uint32_t quantize8_fast(const uint4 hv, float inv) {
+  const uint32_t w[4] = {hv.x, hv.y, hv.z, hv.w};
+  uint32_t packed = 0;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const uint32_t word = w[e >> 1];
+    const float f = (e & 1) ? bf16_hi_f32(word) : bf16_lo_f32(word);
+    const float u = __fadd_rn(__fmul_rn(f, inv), 12582912.0f);
+    packed |= (__float_as_uint(u) & 0xFu) << (4 * e);
+  }
+  return packed;
+}
+
+template <int R, int T, int Dc, bool F32OUT>
+__global__ void __launch_bounds__(kRfThreads, 1)
+boundary_cluster_rf_kernel(const bf16* __restrict__ x, const bf16* __restrict__ res,
+                           const uint4* __restrict__ Uf, const uint4* __restrict__ Vf, int N,
+                           int D, void* __restrict__ h_out, uint8_t* __restrict__ q_out,
+                           float* __restrict__ scale_out) {
+  using C = RfCfg<R, T, Dc>;
+  constexpr int S = C::S, RP = C::RP;
+  constexpr uint32_t pitch = C::pitch;
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, q4 = lane & 3;
+  const uint32_t crank = cluster_ctarank();
+  const uint32_t csize = static_cast<uint32_t>(D / Dc);
+  const int col0 = static_cast<int>(crank) * Dc;
+  const uint32_t cid = cluster_id_x(), ncl = ncluster_x();
+  const int ntiles = (N + T - 1) / T;
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bars = sbase + C::oBars;   // full_res[s] = bars + 8s, full_x[s] = bars + 8(S+s)
+
+  if (tid == 0) {
+    for (int i = 0; i < 2 * S; ++i) mbar_init(bars + 8 * i, 1);
+    fence_mbarrier_init();
+  }
+  __syncthreads();
+
+  // Warp 0: bulk-copy the residual (which = 0) or x (which = 1) rows of loop
+  // iteration `it` into stage it % S.
+  auto issue = [&](int it, int which) {
+    const int tile = static_cast<int>(cid) + it * static_cast<int>(ncl);
+    if (warp != 0 || tile >= ntiles) return;
+    const int s = it % S;
+    const int row0 = tile * T;
+    const int rows = min(T, N - row0);
+    constexpr uint32_t bytes = Dc * 2;
+    const uint32_t bar = bars + 8 * (which * S + s);
+    const uint32_t dst = sbase + s * C::kStage + which * T * pitch;
+    const bf16* src = which ? x : res;
+    if (lane == 0) mbar_arrive_expect_tx(bar, rows * bytes);
+    __syncwarp();
+    if (lane < rows)
+      bulk_g2s(dst + lane * pitch, src + static_cast<size_t>(row0 + lane) * D + col0, bytes, bar);
+    __syncwarp();
+  };
+  issue(0, 0);
+  issue(0, 1);
+  issue(1, 0);
+  issue(1, 1);
+
+  // Factor fragments, resident for the whole launch.
+  const int wm = warp % C::MT, wk = warp / C::MT;
+  uint32_t ub[C::UREG], vb[C::VREG];
+  {
+    const uint4* up = Uf + (static_cast<size_t>(crank) * C::WK + wk) * (C::UREG / 4) * 32 + lane;
+#pragma unroll
+    for (int ch = 0; ch < C::UREG / 4; ++ch) {
+      const uint4 v = __ldg(up + ch * 32);
+      ub[4 * ch] = v.x; ub[4 * ch + 1] = v.y; ub[4 * ch + 2] = v.z; ub[4 * ch + 3] = v.w;
+    }
+    const uint4* vp = Vf + (static_cast<size_t>(crank) * 8 + warp) * (C::VREG / 4) * 32 + lane;
+#pragma unroll
+    for (int ch = 0; ch < C::VREG / 4; ++ch) {
+      const uint4 v = __ldg(vp + ch * 32);
+      vb[4 * ch] = v.x; vb[4 * ch + 1] = v.y; vb[4 * ch + 2] = v.z; vb[4 * ch + 3] = v.w;
+    }
+  }
+
+  float* part = reinterpret_cast<float*>(smem + C::oPart);
+  float* yfull = part;  // the partials are dead once reduced into ybuf
+  float* ybuf = reinterpret_cast<float*>(smem + C::oYbuf);
+  float* wamax = reinterpret_cast<float*>(smem + C::oWamax);
+  float* am2 = reinterpret_cast<float*>(smem + C::oAm2);
+  float* amaxbuf = reinterpret_cast<float*>(smem + C::oAmax);
+  float* rowinv = reinterpret_cast<float*>(smem + C::oRinv);
+
+  for (int it = 0;; ++it) {
+    const int tile = static_cast<int>(cid) + it * static_cast<int>(ncl);
+    if (tile >= ntiles) break;
+    const int s = it % S;
+    const uint32_t par = static_cast<uint32_t>(it / S) & 1u;
+    const int row0 = tile * T;
+    const uint32_t rs = sbase + s * C::kStage;
+    const uint8_t* rs_ptr = smem + s * C::kStage;
+    uint8_t* xs_ptr = smem + s * C::kStage + T * pitch;
+
+    // ---- phase 1: this CTA's partial y = residual[:, slice] U_slice
+    mbar_wait(bars + 8 * s, par, kSiteBoundaryLoad);
+    {
+      float acc[C::NPW][4];
+#pragma unroll
+      for (int p = 0; p < C::NPW; ++p) acc[p][0] = acc[p][1] = acc[p][2] = acc[p][3] = 0.f;
+      const uint32_t a_base = rs + (wm * 16 + (lane & 15)) * pitch + (lane >> 4) * 16;
+#pragma unroll
+      for (int j = 0; j < C::KPW; ++j) {
+        uint32_t a[4];
+        ldmatrix_x4(a_base + (wk * C::KPW + j) * 32, a[0], a[1], a[2], a[3]);
+#pragma unroll
+        for (int p = 0; p < C::NPW; ++p)
+          mma_bf16_16816(acc[p], a, ub[(j * C::NPW + p) * 2], ub[(j * C::NPW + p) * 2 + 1]);
+      }
+      float* pw = part + wk * T * RP;
+#pragma unroll
+      for (int p = 0; p < C::NPW; ++p) {
+        const int col = p * 8 + 2 * q4, row = wm * 16 + g;
+        *reinterpret_cast<float2*>(&pw[row * RP + col]) = make_float2(acc[p][0], acc[p][1]);
+        *reinterpret_cast<float2*>(&pw[(row + 8) * RP + col]) = make_float2(acc[p][2], acc[p][3]);
+      }
+    }
+    __syncthreads();
+    if (tid < T * R / 4) {
+      const int e = 4 * tid, row = e / R, col = e % R;
+      float4 sum = *reinterpret_cast<const float4*>(&part[row * RP + col]);
+#pragma unroll
+      for (int w = 1; w < C::WK; ++w) {
+        const float4 v = *reinterpret_cast<const float4*>(&part[(w * T + row) * RP + col]);
+        sum.x += v.x; sum.y += v.y; sum.z += v.z; sum.w += v.w;
+      }
+      *reinterpret_cast<float4*>(&ybuf[e]) = sum;
+    }
+
+    // ---- y over the cluster; warp 0 stages the residual rows of iteration
+    // it+2 meanwhile (its stage was released at the end of iteration it-1)
+    cluster_arrive();
+    issue(it + 2, 0);
+    cluster_wait();
+    if (tid < T * R / 4) {
+      const int e = 4 * tid, row = e / R, col = e % R;
+      *reinterpret_cast<float4*>(&yfull[row * RP + col]) =
+          cluster_sum_f32x4(sbase + C::oYbuf + 16u * tid, csize);
+    }
+    __syncthreads();
+
+    // ---- phase 2: h = (res + x) + y V_slice^T, bf16 round, row amax
+    mbar_wait(bars + 8 * (S + s), par, kSiteBoundaryLoad);
+    {
+      uint32_t ahi[C::MT][C::KS2][4], alo[C::MT][C::KS2][4];
+#pragma unroll
+      for (int mt = 0; mt < C::MT; ++mt)
+#pragma unroll
+        for (int ks = 0; ks < C::KS2; ++ks) {
+          const int r0 = mt * 16 + g, c0 = ks * 16 + 2 * q4;
+          split_bf16x2(*reinterpret_cast<const float2*>(&yfull[r0 * RP + c0]), ahi[mt][ks][0], alo[mt][ks][0]);
+          split_bf16x2(*reinterpret_cast<const float2*>(&yfull[(r0 + 8) * RP + c0]), ahi[mt][ks][1], alo[mt][ks][1]);
+          split_bf16x2(*reinterpret_cast<const float2*>(&yfull[r0 * RP + c0 + 8]), ahi[mt][ks][2], alo[mt][ks][2]);
+          split_bf16x2(*reinterpret_cast<const float2*>(&yfull[(r0 + 8) * RP + c0 + 8]), ahi[mt][ks][3], alo[mt][ks][3]);
+        }
+      __nv_bfloat162 rmax2[C::MT];   // .x: row mt*16+g, .y: row mt*16+g+8
+#pragma unroll
+      for (int mt = 0; mt < C::MT; ++mt) rmax2[mt] = __float2bfloat162_rn(0.f);
+#pragma unroll
+      for (int t = 0; t < C::NTW; ++t) {
+        const int d0 = (warp * C::NTW + t) * 8;
+#pragma unroll
+        for (int mt = 0; mt < C::MT; ++mt) {
+          const int rowA = mt * 16 + g;
+          const uint32_t offA = rowA * pitch + (d0 + 2 * q4) * 2;
+          const uint32_t offB = offA + 8 * pitch;
+          const uint32_t rA = *reinterpret_cast<const uint32_t*>(rs_ptr + offA);
+          const uint32_t xA = *reinterpret_cast<const uint32_t*>(xs_ptr + offA);
+          const uint32_t rB = *reinterpret_cast<const uint32_t*>(rs_ptr + offB);
+          const uint32_t xB = *reinterpret_cast<const uint32_t*>(xs_ptr + offB);
+          // accumulators start at residual + x; the tensor cores add y V^T
+          float acc[4] = {bf16_lo_f32(rA) + bf16_lo_f32(xA), bf16_hi_f32(rA) + bf16_hi_f32(xA),
+                          bf16_lo_f32(rB) + bf16_lo_f32(xB), bf16_hi_f32(rB) + bf16_hi_f32(xB)};
+#pragma unroll
+          for (int ks = 0; ks < C::KS2; ++ks) {
+            const uint32_t b0 = vb[(t * C::KS2 + ks) * 2], b1 = vb[(t * C::KS2 + ks) * 2 + 1];
+            mma_bf16_16816(acc, ahi[mt][ks], b0, b1);
+            mma_bf16_16816(acc, alo[mt][ks], b0, b1);
+          }
+          const __nv_bfloat162 hA = __floats2bfloat162_rn(acc[0], acc[1]);
+          const __nv_bfloat162 hB = __floats2bfloat162_rn(acc[2], acc[3]);
+          *reinterpret_cast<__nv_bfloat162*>(xs_ptr + offA) = hA;
+          *reinterpret_cast<__nv_bfloat162*>(xs_ptr + offB) = hB;
+          const __nv_bfloat162 mA = __habs2(hA), mB = __habs2(hB);
+          rmax2[mt] = __hmax2(rmax2[mt],
+                              __halves2bfloat162(__hmax(__low2bfloat16(mA), __high2bfloat16(mA)),
+                                                 __hmax(__low2bfloat16(mB), __high2bfloat16(mB))));
+          if constexpr (F32OUT) {
+            if (h_out != nullptr) {
+              float* hf = static_cast<float*>(h_out) + col0 + d0 + 2 * q4;
+              if (row0 + rowA < N)
+                *reinterpret_cast<float2*>(hf + static_cast<size_t>(row0 + rowA) * D) = make_float2(acc[0], acc[1]);
+              if (row0 + rowA + 8 < N)
+                *reinterpret_cast<float2*>(hf + static_cast<size_t>(row0 + rowA + 8) * D) = make_float2(acc[2], acc[3]);
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int mt = 0; mt < C::MT; ++mt) {
+        float mA = __bfloat162float(__low2bfloat16(rmax2[mt]));
+        float mB = __bfloat162float(__high2bfloat16(rmax2[mt]));
+        mA = fmaxf(mA, __shfl_xor_sync(0xffffffffu, mA, 1));
+        mA = fmaxf(mA, __shfl_xor_sync(0xffffffffu, mA, 2));
+        mB = fmaxf(mB, __shfl_xor_sync(0xffffffffu, mB, 1));
+        mB = fmaxf(mB, __shfl_xor_sync(0xffffffffu, mB, 2));
+        if (q4 == 0) {
+          wamax[warp * T + mt * 16 + g] = mA;
+          wamax[warp * T + mt * 16 + g + 8] = mB;
+        }
+      }
+      __syncthreads();
+      if (tid < T) {
+        float m = 0.f;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) m = fmaxf(m, wamax[w * T + tid]);
+        amaxbuf[tid] = m;
+      }
+    }
+
+    // ---- amax over the cluster (warp 0 stages the x rows of iteration it+2)
+    cluster_arrive();
+    issue(it + 2, 1);
+    cluster_wait();
+    for (int i = tid; i < static_cast<int>(csize) * T; i += kRfThreads)
+      am2[i] = ld_dsmem_f32(map_to_rank(sbase + C::oAmax + 4u * (i % T), static_cast<uint32_t>(i / T)));
+    __syncthreads();
+    if (tid < T) {
+      float m = 0.f;
+      for (uint32_t c = 0; c < csize; ++c) m = fmaxf(m, am2[c * T + tid]);
+      float inv, sc;
+      inv_and_scale(m, inv, sc);
+      rowinv[tid] = inv;
+      if (crank == 0 && row0 + tid < N) scale_out[row0 + tid] = sc;
+    }
+    __syncthreads();
+
+    // ---- h' (bf16) and packed codes of this CTA's slice
+    {
+      constexpr int vpr = Dc / 8;
+#pragma unroll 4
+      for (int i = tid; i < T * vpr; i += kRfThreads) {
+        const int row = i / vpr, v = i % vpr;
+        if (row0 + row >= N) continue;
+        const uint4 hv = *reinterpret_cast<const uint4*>(xs_ptr + row * pitch + v * 16);
+        const size_t gi = static_cast<size_t>(row0 + row) * D + col0 + v * 8;
+        if constexpr (!F32OUT) {
+          if (h_out != nullptr) *reinterpret_cast<uint4*>(static_cast<bf16*>(h_out) + gi) = hv;
+        }
+        *reinterpret_cast<uint32_t*>(q_out + gi / 2) = quantize8_fast(hv, rowinv[row]);
+      }
+    }
+    // This stage is refilled by bulk copies during the next iteration: order
+    // the generic-proxy accesses above before those async-proxy writes (the
+    // first CTA barrier of the next iteration completes the hand-off).
+    fence_proxy_async_smem();
+  }
+  // No CTA may leave while a peer can still read its shared memory.
+  cluster_sync();
+}
+
+// ============================================================================
+// Shared-memory-resident factors (r = 64, 128), 2-stage tile ring.
+// ============================================================================
+
+template <int T, int R>
+struct SmemCfg {
+  static constexpr int kWarps = kBoundaryThreads / 32;
+  static constexpr int MT = T / 16;                       // m16 tiles per token tile
+  static constexpr int NT1 = R / 8;                       // n8 tiles of y
+  static constexpr int WN = (NT1 / 4) > 1 ? NT1 / 4 : 1;  // warps along r (phase 1)
+  static constexpr int WK = kWarps / (MT * WN);           // warps along Dc (phase 1)
+  static constexpr int NPW = NT1 / WN;                    // n8 tiles per warp (2 or 4)
+  static constexpr int KS2 = R / 16;                      // k16 steps of phase 2
+  static constexpr int CPR = R / 8;                       // 16-byte chunks per V row
+  static constexpr int VL = (8 / CPR) > 1 ? 8 / CPR : 1;  // V rows per 128-byte line
+  static constexpr int VXM = (CPR < 8 ? CPR : 8) - 1;     // chunk swizzle mask
+  static constexpr int RP = R + 8;                        // padded fp32 row
+  static_assert(T == 16 || T == 32, "token tile");
+  static_assert(R == 16 || R == 32 || R == 64 || R == 128, "padded rank");
+  static_assert(MT * WN * WK == kWarps, "warp split");
+  static_assert(NPW == 2 || NPW == 4, "phase-1 n tiles per warp");
+};
+
+// Shared-memory carve-up of the shared-memory-factor kernel (host and device).
+struct BoundarySmem {
+  uint32_t us, vs, stage0, stage_bytes, partial, ybuf, wamax, am2, amaxbuf, rowinv, bars, total;
+};
+
+__host__ __device__ inline BoundarySmem boundary_smem_layout(int T, int R, int Dc) {
+  const int MT = T / 16, NT1 = R / 8;
+  const int WN = (NT1 / 4) > 1 ? NT1 / 4 : 1;
+  const int WK = 8 / (MT * WN);
+  const int RP = R + 8;
+  const uint32_t pitch = static_cast<uint32_t>(Dc) * 2 + 16;
+  BoundarySmem L;
+  uint32_t off = 0;
+  L.us = off;          off += R * pitch;                          // U^T slice, padded rows
+  L.vs = off;          off += static_cast<uint32_t>(Dc) * R * 2;  // V slice, swizzled
+  L.stage0 = off;      L.stage_bytes = 2 * T * pitch;  off += 2 * L.stage_bytes;
+  L.partial = off;     off += WK * T * RP * 4;                    // y (padded) aliases [0]
+  L.ybuf = off;        off += T * R * 4;
+  L.wamax = off;       off += 8 * T * 4;
+  L.am2 = off;         off += 16 * T * 4;
+  L.amaxbuf = off;     off += T * 4;
+  L.rowinv = off;      off += T * 4;
+  off = (off + 15u) & ~15u;
+  L.bars = off;        off += 4 * 8;
+  L.total = off;
+  return L;
+}
+
 template <int T, int R, bool F32OUT>
 __global__ void __launch_bounds__(kBoundaryThreads, 1)
-boundary_cluster_kernel(const bf16* __restrict__ x, const bf16* __restrict__ res,
-                        const bf16* __restrict__ Ut,   // [R, D]  (U transposed, zero padded)
-                        const bf16* __restrict__ V,    // [D, R]  (zero padded)
-                        int N, int D, int Dc, void* __restrict__ h_out,
-                        uint8_t* __restrict__ q_out, float* __restrict__ scale_out) {
-  using C = BoundaryCfg<T, R>;
+boundary_cluster_smem_kernel(const bf16* __restrict__ x, const bf16* __restrict__ res,
+                             const bf16* __restrict__ Ut,   // [R, D]  (U transposed, zero padded)
+                             const bf16* __restrict__ V,    // [D, R]  (zero padded)
+                             int N, int D, int Dc, void* __restrict__ h_out,
+                             uint8_t* __restrict__ q_out, float* __restrict__ scale_out) {
+  using C = SmemCfg<T, R>;
+  constexpr int RP = C::RP;
   extern __shared__ __align__(128) uint8_t smem[];
   const BoundarySmem L = boundary_smem_layout(T, R, Dc);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -128,36 +572,22 @@ boundary_cluster_kernel(const bf16* __restrict__ x, const bf16* __restrict__ res
   const int ntiles = (N + T - 1) / T;
   const uint32_t pitch = static_cast<uint32_t>(Dc) * 2 + 16;
   const uint32_t sbase = smem_u32(smem);
-  const uint32_t bar_res0 = sbase + L.bars, bar_x0 = sbase + L.bars + 16;
+  const uint32_t bars = sbase + L.bars;
 
   if (tid == 0) {
-    for (int i = 0; i < 4; ++i) mbar_init(sbase + L.bars + 8 * i, 1);
+    for (int i = 0; i < 4; ++i) mbar_init(bars + 8 * i, 1);
     fence_mbarrier_init();
   }
   __syncthreads();
 
-  // Stage the residual and x tiles of loop iteration `it` (warp 0 only).
   auto issue = [&](int it) {
     const int tile = static_cast<int>(cid) + it * static_cast<int>(ncl);
     if (tile >= ntiles || warp != 0) return;
-    const int row0 = tile * T;
-    const int rows = min(T, N - row0);
     const int s = it & 1;
-    const uint32_t bytes = static_cast<uint32_t>(Dc) * 2;
-    if (lane == 0) {
-      mbar_arrive_expect_tx(bar_res0 + 8 * s, rows * bytes);
-      mbar_arrive_expect_tx(bar_x0 + 8 * s, rows * bytes);
-    }
-    __syncwarp();
-    if (lane < rows) {
-      const size_t gofs = static_cast<size_t>(row0 + lane) * D + col0;
-      const uint32_t rdst = sbase + (s ? L.stage[1][0] : L.stage[0][0]) + lane * pitch;
-      const uint32_t xdst = sbase + (s ? L.stage[1][1] : L.stage[0][1]) + lane * pitch;
-      bulk_g2s(rdst, res + gofs, bytes, bar_res0 + 8 * s);
-      bulk_g2s(xdst, x + gofs, bytes, bar_x0 + 8 * s);
-    }
+    const uint32_t st = sbase + L.stage0 + s * L.stage_bytes;
+    stage_tile(x, res, tile * T, N, D, col0, Dc, T, st, st + T * pitch, pitch, bars + 16 * s,
+               bars + 16 * s + 8, lane);
   };
-
   issue(0);
   issue(1);
 
@@ -179,9 +609,10 @@ boundary_cluster_kernel(const bf16* __restrict__ x, const bf16* __restrict__ res
   __syncthreads();
 
   float* part = reinterpret_cast<float*>(smem + L.partial);
+  float* yfull = part;
   float* ybuf = reinterpret_cast<float*>(smem + L.ybuf);
-  float* yfull = reinterpret_cast<float*>(smem + L.yfull);
   float* wamax = reinterpret_cast<float*>(smem + L.wamax);
+  float* am2 = reinterpret_cast<float*>(smem + L.am2);
   float* amaxbuf = reinterpret_cast<float*>(smem + L.amaxbuf);
   float* rowinv = reinterpret_cast<float*>(smem + L.rowinv);
 
@@ -191,14 +622,12 @@ boundary_cluster_kernel(const bf16* __restrict__ x, const bf16* __restrict__ res
     const int s = it & 1;
     const uint32_t par = static_cast<uint32_t>(it >> 1) & 1u;
     const int row0 = tile * T;
-    const uint32_t rs_off = s ? L.stage[1][0] : L.stage[0][0];
-    const uint32_t xs_off = s ? L.stage[1][1] : L.stage[0][1];
-    const uint32_t rs = sbase + rs_off;
-    uint8_t* xs_ptr = smem + xs_off;
-    const uint8_t* rs_ptr = smem + rs_off;
+    const uint32_t rs = sbase + L.stage0 + s * L.stage_bytes;
+    const uint8_t* rs_ptr = smem + L.stage0 + s * L.stage_bytes;
+    uint8_t* xs_ptr = smem + L.stage0 + s * L.stage_bytes + T * pitch;
 
     // ---- phase 1: partial y = residual_tile[:, slice] * U_slice (tensor cores)
-    mbar_wait(bar_res0 + 8 * s, par, kSiteBoundaryLoad);
+    mbar_wait(bars + 16 * s, par, kSiteBoundaryLoad);
     {
       const int wm = warp % C::MT;
       const int wn = (warp / C::MT) % C::WN;
@@ -223,40 +652,38 @@ boundary_cluster_kernel(const bf16* __restrict__ x, const bf16* __restrict__ res
           mma_bf16_16816(acc[2 * p + 1], a, b2, b3);
         }
       }
-      float* pw = part + wk * T * R;
+      float* pw = part + wk * T * RP;
 #pragma unroll
       for (int j = 0; j < C::NPW; ++j) {
         const int col = (wn * C::NPW + j) * 8 + 2 * q4;
         const int row = wm * 16 + g;
-        *reinterpret_cast<float2*>(&pw[row * R + col]) = make_float2(acc[j][0], acc[j][1]);
-        *reinterpret_cast<float2*>(&pw[(row + 8) * R + col]) = make_float2(acc[j][2], acc[j][3]);
+        *reinterpret_cast<float2*>(&pw[row * RP + col]) = make_float2(acc[j][0], acc[j][1]);
+        *reinterpret_cast<float2*>(&pw[(row + 8) * RP + col]) = make_float2(acc[j][2], acc[j][3]);
       }
     }
     __syncthreads();
-    for (int i = tid * 4; i < T * R; i += kBoundaryThreads * 4) {
-      float4 sum = *reinterpret_cast<const float4*>(&part[i]);
+    for (int e = tid * 4; e < T * R; e += kBoundaryThreads * 4) {
+      const int row = e / R, col = e % R;
+      float4 sum = *reinterpret_cast<const float4*>(&part[row * RP + col]);
 #pragma unroll
       for (int w = 1; w < C::WK; ++w) {
-        const float4 v = *reinterpret_cast<const float4*>(&part[w * T * R + i]);
+        const float4 v = *reinterpret_cast<const float4*>(&part[(w * T + row) * RP + col]);
         sum.x += v.x; sum.y += v.y; sum.z += v.z; sum.w += v.w;
       }
-      *reinterpret_cast<float4*>(&ybuf[i]) = sum;
+      *reinterpret_cast<float4*>(&ybuf[e]) = sum;
     }
 
-    // ---- cluster reduction of y (same order in every CTA -> identical y)
+    // ---- y over the cluster
     cluster_sync();
-    {
-      const uint32_t yb = sbase + L.ybuf;
-      for (int i = tid; i < T * R; i += kBoundaryThreads) {
-        float sum = 0.f;
-        for (uint32_t c = 0; c < csize; ++c) sum += ld_dsmem_f32(map_to_rank(yb, c) + 4u * i);
-        yfull[i] = sum;
-      }
+    for (int e = tid * 4; e < T * R; e += kBoundaryThreads * 4) {
+      const int row = e / R, col = e % R;
+      *reinterpret_cast<float4*>(&yfull[row * RP + col]) =
+          cluster_sum_f32x4(sbase + L.ybuf + 4u * e, csize);
     }
     __syncthreads();
 
     // ---- phase 2: h = (res + x) + y V_slice^T, bf16 round, row amax
-    mbar_wait(bar_x0 + 8 * s, par, kSiteBoundaryLoad);
+    mbar_wait(bars + 16 * s + 8, par, kSiteBoundaryLoad);
     {
       uint32_t ahi[C::MT][C::KS2][4], alo[C::MT][C::KS2][4];
 #pragma unroll
@@ -264,18 +691,10 @@ boundary_cluster_kernel(const bf16* __restrict__ x, const bf16* __restrict__ res
 #pragma unroll
         for (int ks = 0; ks < C::KS2; ++ks) {
           const int r0 = mt * 16 + g, c0 = ks * 16 + 2 * q4;
-          const float2 v[4] = {*reinterpret_cast<const float2*>(&yfull[r0 * R + c0]),
-                               *reinterpret_cast<const float2*>(&yfull[(r0 + 8) * R + c0]),
-                               *reinterpret_cast<const float2*>(&yfull[r0 * R + c0 + 8]),
-                               *reinterpret_cast<const float2*>(&yfull[(r0 + 8) * R + c0 + 8])};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const __nv_bfloat162 hi = __floats2bfloat162_rn(v[e].x, v[e].y);
-            const float2 hf = __bfloat1622float2(hi);
-            const __nv_bfloat162 lo = __floats2bfloat162_rn(v[e].x - hf.x, v[e].y - hf.y);
-            ahi[mt][ks][e] = *reinterpret_cast<const uint32_t*>(&hi);
-            alo[mt][ks][e] = *reinterpret_cast<const uint32_t*>(&lo);
-          }
+          split_bf16x2(*reinterpret_cast<const float2*>(&yfull[r0 * RP + c0]), ahi[mt][ks][0], alo[mt][ks][0]);
+          split_bf16x2(*reinterpret_cast<const float2*>(&yfull[(r0 + 8) * RP + c0]), ahi[mt][ks][1], alo[mt][ks][1]);
+          split_bf16x2(*reinterpret_cast<const float2*>(&yfull[r0 * RP + c0 + 8]), ahi[mt][ks][2], alo[mt][ks][2]);
+          split_bf16x2(*reinterpret_cast<const float2*>(&yfull[(r0 + 8) * RP + c0 + 8]), ahi[mt][ks][3], alo[mt][ks][3]);
         }
       float rmax[C::MT][2];
 #pragma unroll
@@ -306,79 +725,21 @@ boundary_cluster_kernel(const bf16* __restrict__ x, const bf16* __restrict__ res
             mma_bf16_16816(acc, ahi[mt][ks], b[ks][0], b[ks][1]);
             mma_bf16_16816(acc, alo[mt][ks], b[ks][0], b[ks][1]);
           }
-#pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            const int row = mt * 16 + g + 8 * hh;
-            const uint32_t off = row * pitch + (d0 + 2 * q4) * 2;
-            const uint32_t rw = *reinterpret_cast<const uint32_t*>(rs_ptr + off);
-            const uint32_t xw = *reinterpret_cast<const uint32_t*>(xs_ptr + off);
-            const float h0 = (bf16_lo_f32(rw) + bf16_lo_f32(xw)) + acc[2 * hh];
-            const float h1 = (bf16_hi_f32(rw) + bf16_hi_f32(xw)) + acc[2 * hh + 1];
-            const uint32_t hb = pack_bf16x2(h0, h1);
-            *reinterpret_cast<uint32_t*>(xs_ptr + off) = hb;
-            rmax[mt][hh] = fmaxf(rmax[mt][hh], fmaxf(fabsf(bf16_lo_f32(hb)), fabsf(bf16_hi_f32(hb))));
-            if constexpr (F32OUT) {
-              if (h_out != nullptr && row0 + row < N) {
-                float* hf = static_cast<float*>(h_out) +
-                            static_cast<size_t>(row0 + row) * D + col0 + d0 + 2 * q4;
-                *reinterpret_cast<float2*>(hf) = make_float2(h0, h1);
-              }
-            }
-          }
+          finish_n8<F32OUT>(acc, rs_ptr, xs_ptr, pitch, mt * 16 + g, d0 + 2 * q4, rmax[mt], h_out, row0,
+                            N, D, col0);
         }
       }
-#pragma unroll
-      for (int mt = 0; mt < C::MT; ++mt)
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          float m = rmax[mt][hh];
-          m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
-          m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
-          if (q4 == 0) wamax[warp * T + mt * 16 + g + 8 * hh] = m;
-        }
-    }
-    __syncthreads();
-    if (tid < T) {
-      float m = 0.f;
-#pragma unroll
-      for (int w = 0; w < 8; ++w) m = fmaxf(m, wamax[w * T + tid]);
-      amaxbuf[tid] = m;
+      publish_amax<C::MT, T>(rmax, wamax, amaxbuf, warp, lane, tid);
     }
 
-    // ---- cluster reduction of the row amax
+    // ---- amax over the cluster, then codes
     cluster_sync();
-    if (tid < T) {
-      const uint32_t ab = sbase + L.amaxbuf + 4u * tid;
-      float m = 0.f;
-      for (uint32_t c = 0; c < csize; ++c) m = fmaxf(m, ld_dsmem_f32(map_to_rank(ab, c)));
-      float inv, sc;
-      inv_and_scale(m, inv, sc);
-      rowinv[tid] = inv;
-      if (crank == 0 && row0 + tid < N) scale_out[row0 + tid] = sc;
-    }
-    __syncthreads();
-
-    // ---- store h' (bf16) and the packed codes of this CTA's slice
-    {
-      const int vpr = Dc / 8;
-      for (int i = tid; i < T * vpr; i += kBoundaryThreads) {
-        const int row = i / vpr, v = i % vpr;
-        if (row0 + row >= N) continue;
-        const uint4 hv = *reinterpret_cast<const uint4*>(xs_ptr + row * pitch + v * 16);
-        const size_t gi = static_cast<size_t>(row0 + row) * D + col0 + v * 8;
-        if constexpr (!F32OUT) {
-          if (h_out != nullptr) *reinterpret_cast<uint4*>(static_cast<bf16*>(h_out) + gi) = hv;
-        }
-        *reinterpret_cast<uint32_t*>(q_out + gi / 2) = quantize8(hv, rowinv[row]);
-      }
-    }
-    // This stage is refilled by bulk copies next: order the generic-proxy
-    // writes above before those async-proxy writes.
+    gather_amax<T>(sbase + L.amaxbuf, am2, rowinv, scale_out, csize, crank, row0, N, tid);
+    store_tile<F32OUT>(xs_ptr, pitch, rowinv, T, Dc, row0, N, D, col0, h_out, q_out, tid);
     fence_proxy_async_smem();
     __syncthreads();
     issue(it + 2);
   }
-  // No CTA may leave while a peer can still read its shared memory.
   cluster_sync();
 }
 
@@ -449,6 +810,46 @@ boundary_rowwise_kernel(const bf16* __restrict__ x, const bf16* __restrict__ res
     }
     __syncthreads();
   }
+}
+
+// Fragment-ordered factor copies for boundary_cluster_rf_kernel<R, T, Dc>,
+// built on the host by the plan. `Ub`/`Vb` are the bf16 bit patterns of U and
+// V, [D, R] row-major (R = padded rank). Output: arrays of 32-bit words in the
+// order the kernel loads them: for CTA c and phase-1 warp group wk, register
+// i = (j*NPW + p)*2 + e of lane (g, q) holds (U[d][n], U[d+1][n]) with
+// d = c*Dc + (wk*KPW + j)*16 + 2q + 8e and n = 8p + g; for compute warp w,
+// register i = (t*KS2 + k)*2 + e holds (V[d][m], V[d][m+1]) with
+// d = c*Dc + (w*NTW + t)*8 + g and m = 16k + 2q + 8e.
+inline void rf_pack_factors(const uint16_t* Ub, const uint16_t* Vb, int D, int R, int T, int Dc,
+                            uint32_t* Uf, uint32_t* Vf) {
+  const int MT = T / 16, WK = 8 / MT, KPW = Dc / 16 / WK, NPW = R / 8, KS2 = R / 16, NTW = Dc / 64;
+  const int UREG = KPW * NPW * 2, VREG = NTW * KS2 * 2;
+  const int C = D / Dc;
+  auto pair = [](uint16_t lo, uint16_t hi) { return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16); };
+  for (int c = 0; c < C; ++c)
+    for (int wk = 0; wk < WK; ++wk)
+      for (int lane = 0; lane < 32; ++lane) {
+        const int g = lane >> 2, q = lane & 3;
+        for (int i = 0; i < UREG; ++i) {
+          const int e = i & 1, p = (i >> 1) % NPW, j = (i >> 1) / NPW;
+          const int d = c * Dc + (wk * KPW + j) * 16 + 2 * q + 8 * e;
+          const int n = p * 8 + g;
+          const size_t idx = ((static_cast<size_t>(c * WK + wk) * (UREG / 4) + i / 4) * 32 + lane) * 4 + i % 4;
+          Uf[idx] = pair(Ub[static_cast<size_t>(d) * R + n], Ub[static_cast<size_t>(d + 1) * R + n]);
+        }
+      }
+  for (int c = 0; c < C; ++c)
+    for (int w = 0; w < 8; ++w)
+      for (int lane = 0; lane < 32; ++lane) {
+        const int g = lane >> 2, q = lane & 3;
+        for (int i = 0; i < VREG; ++i) {
+          const int e = i & 1, k = (i >> 1) % KS2, t = (i >> 1) / KS2;
+          const int d = c * Dc + (w * NTW + t) * 8 + g;
+          const int m = k * 16 + 2 * q + 8 * e;
+          const size_t idx = ((static_cast<size_t>(c * 8 + w) * (VREG / 4) + i / 4) * 32 + lane) * 4 + i % 4;
+          Vf[idx] = pair(Vb[static_cast<size_t>(d) * R + m], Vb[static_cast<size_t>(d) * R + m + 1]);
+        }
+      }
 }
 
 }  // namespace respin

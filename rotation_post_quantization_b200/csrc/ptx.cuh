@@ -17,7 +17,9 @@ enum StatusSite : int {
   kSiteBoundaryLoad = 101,   // boundary kernel: waiting for a staged tile
   kSiteGemmEmpty = 201,      // GEMM producer: waiting for a free stage
   kSiteGemmFull = 202,       // GEMM MMA warp: waiting for a filled stage
-  kSiteGemmAccum = 203,      // GEMM epilogue: waiting for the accumulator
+  kSiteGemmAccum = 203,      // GEMM epilogue / MMA: waiting for an accumulator buffer
+  kSiteGemmPackedFull = 204, // GEMM producer: waiting for a packed K block (TMA)
+  kSiteGemmPackedEmpty = 205,// GEMM TMA warp: waiting for a free packed stage
 };
 
 // Upper bound on any single wait inside a kernel (nanoseconds of globaltimer).
@@ -110,6 +112,18 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
       : "memory");
 }
 
+// 2-D tensor copy global -> shared through a tensor map (tile mode, no
+// multicast). (x, y) is the box origin in elements; x * element size must be
+// a multiple of 16 bytes. Out-of-range elements are zero filled and counted.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, int x, int y,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(tmap), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+
 // ---------------------------------------------------------------- clusters
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {
@@ -137,6 +151,21 @@ __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
+// Split cluster barrier: arrive (release) now, wait (acquire) later; work
+// placed between the two overlaps the barrier latency.
+__device__ __forceinline__ void cluster_arrive() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Named CTA barrier over `nthreads` threads (a subset of warps).
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
 // Address of the same shared-memory offset in CTA `rank` of this cluster.
 __device__ __forceinline__ uint32_t map_to_rank(uint32_t addr, uint32_t rank) {
   uint32_t r;
@@ -148,6 +177,30 @@ __device__ __forceinline__ float ld_dsmem_f32(uint32_t addr) {
   float v;
   asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
   return v;
+}
+
+__device__ __forceinline__ float4 ld_dsmem_f32x4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0,%1,%2,%3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+
+// Sum over the cluster of the float4 at byte offset `addr` of every CTA's
+// shared memory, in rank order 0..csize-1 (identical in every CTA). All
+// remote loads are issued before the first addition.
+__device__ __forceinline__ float4 cluster_sum_f32x4(uint32_t addr, uint32_t csize) {
+  float4 v[16];
+#pragma unroll
+  for (uint32_t c = 0; c < 16; ++c)
+    if (c < csize) v[c] = ld_dsmem_f32x4(map_to_rank(addr, c));
+  float4 s = v[0];
+#pragma unroll
+  for (uint32_t c = 1; c < 16; ++c)
+    if (c < csize) { s.x += v[c].x; s.y += v[c].y; s.z += v[c].z; s.w += v[c].w; }
+  return s;
 }
 
 // ---------------------------------------------------------------- warp MMA

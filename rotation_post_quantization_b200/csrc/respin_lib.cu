@@ -2,6 +2,7 @@
 // include/respin.h (argument validation, plans, launch configuration, error
 // reporting). One translation unit holds every kernel so that the device
 // status word is a single symbol without relocatable device code.
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -60,6 +61,7 @@ bool aligned(const void* p, size_t a) {
 // ------------------------------------------------------------ plans
 
 struct BoundaryConfig {
+  bool rf = false;          // register-resident factors (boundary_cluster_rf_kernel)
   int T = 0, R = 0, cluster = 0, Dc = 0;
   size_t smem = 0;
   int max_clusters = 0;
@@ -72,7 +74,7 @@ struct respin_plan_s {
   int D = 0, r = 0, r_pad = 0;
   unsigned flags = 0;
   int device = -1;
-  __nv_bfloat16* factors = nullptr;  // [r_pad, D] U^T then [D, r_pad] V
+  __nv_bfloat16* factors = nullptr;  // 2 * D * r_pad bf16: U part then V part
   BoundaryConfig cfg;
 };
 
@@ -87,22 +89,78 @@ bool plan_alive(respin_plan_s* p) {
 }
 
 template <int T, int R, bool F32>
-const void* cluster_fn() {
-  return reinterpret_cast<const void*>(&boundary_cluster_kernel<T, R, F32>);
+const void* smem_fn() {
+  return reinterpret_cast<const void*>(&boundary_cluster_smem_kernel<T, R, F32>);
 }
 
-const void* pick_cluster_fn(int T, int R, bool f32) {
+const void* pick_smem_fn(int T, int R, bool f32) {
 #define RESPIN_PICK(TT, RR)                                                   \
-  if (T == TT && R == RR) return f32 ? cluster_fn<TT, RR, true>() : cluster_fn<TT, RR, false>();
+  if (T == TT && R == RR) return f32 ? smem_fn<TT, RR, true>() : smem_fn<TT, RR, false>();
   RESPIN_PICK(32, 16) RESPIN_PICK(32, 32) RESPIN_PICK(32, 64)
   RESPIN_PICK(16, 16) RESPIN_PICK(16, 32) RESPIN_PICK(16, 64) RESPIN_PICK(16, 128)
 #undef RESPIN_PICK
   return nullptr;
 }
 
-// Choose cluster size and token tile: the smallest cluster whose per-CTA
-// slice (resident U^T and V slices plus a two-stage residual/x ring) fits in
-// shared memory, preferring 32-token tiles.
+constexpr int kRfT = 16;  // tokens per tile of the register-factor kernel
+
+template <int R, int Dc, bool F32>
+const void* rf_fn() {
+  return reinterpret_cast<const void*>(&boundary_cluster_rf_kernel<R, kRfT, Dc, F32>);
+}
+
+const void* pick_rf_fn(int R, int Dc, bool f32) {
+#define RESPIN_PICK(RR, DD)                                                   \
+  if (R == RR && Dc == DD) return f32 ? rf_fn<RR, DD, true>() : rf_fn<RR, DD, false>();
+  RESPIN_PICK(16, 256) RESPIN_PICK(16, 512) RESPIN_PICK(16, 1024)
+  RESPIN_PICK(32, 256) RESPIN_PICK(32, 512) RESPIN_PICK(32, 1024)
+#undef RESPIN_PICK
+  return nullptr;
+}
+
+size_t rf_smem(int R, int Dc) {
+#define RESPIN_SMEM(RR, DD) \
+  if (R == RR && Dc == DD) return RfCfg<RR, kRfT, DD>::kSmem;
+  RESPIN_SMEM(16, 256) RESPIN_SMEM(16, 512) RESPIN_SMEM(16, 1024)
+  RESPIN_SMEM(32, 256) RESPIN_SMEM(32, 512) RESPIN_SMEM(32, 1024)
+#undef RESPIN_SMEM
+  return 0;
+}
+
+// Largest number of co-resident clusters of `C` CTAs for kernel `fn`
+// (0 if the configuration cannot be launched).
+int max_active_clusters(const void* fn, int C, size_t smem, int threads) {
+  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  if (C > 8 && cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  cudaLaunchConfig_t lc = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  lc.gridDim = dim3(C, 1, 1);
+  lc.blockDim = dim3(threads, 1, 1);
+  lc.dynamicSmemBytes = smem;
+  lc.attrs = attr;
+  lc.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, fn, &lc) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  return n;
+}
+
+// Choose the boundary kernel. r <= 32: register-resident factors with 512
+// (else 256) columns per CTA. Otherwise: shared-memory factors, the smallest
+// cluster whose per-CTA slice fits, preferring 32-token tiles.
 respin_status_t configure_boundary(int D, int R, bool f32, BoundaryConfig* out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -110,40 +168,34 @@ respin_status_t configure_boundary(int D, int R, bool f32, BoundaryConfig* out) 
   int smem_optin = 0;
   e = cudaDeviceGetAttribute(&smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
-  const int clusters[] = {1, 2, 4, 8, 16};
-  const int tiles[] = {32, 16};
-  for (int C : clusters) {
+  if (R <= 32) {
+    for (int Dc : {1024, 512, 256}) {
+      if (D % Dc || D / Dc > 16) continue;
+      const int C = D / Dc;
+      const size_t smem = rf_smem(R, Dc);
+      if (smem == 0 || smem > static_cast<size_t>(smem_optin)) continue;
+      const void* fn = pick_rf_fn(R, Dc, f32);
+      const int n = max_active_clusters(fn, C, smem, kRfThreads);
+      if (n <= 0) continue;
+      out->rf = true; out->T = kRfT; out->R = R; out->cluster = C; out->Dc = Dc;
+      out->smem = smem; out->max_clusters = n; out->fn = fn;
+      return ok();
+    }
+  }
+  for (int C : {1, 2, 4, 8, 16}) {
     if (D % C) continue;
     const int Dc = D / C;
     if (Dc % 64) continue;
-    for (int T : tiles) {
+    for (int T : {32, 16}) {
       if (T * R > 2048) continue;
-      const void* fn = pick_cluster_fn(T, R, f32);
+      const void* fn = pick_smem_fn(T, R, f32);
       if (!fn) continue;
       const size_t smem = boundary_smem_layout(T, R, Dc).total;
       if (smem > static_cast<size_t>(smem_optin)) continue;
-      e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(smem)");
-      if (C > 8) {
-        e = cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-        if (e != cudaSuccess) { cudaGetLastError(); continue; }
-      }
-      cudaLaunchConfig_t lc = {};
-      cudaLaunchAttribute attr[1];
-      attr[0].id = cudaLaunchAttributeClusterDimension;
-      attr[0].val.clusterDim.x = C;
-      attr[0].val.clusterDim.y = 1;
-      attr[0].val.clusterDim.z = 1;
-      lc.gridDim = dim3(C, 1, 1);
-      lc.blockDim = dim3(kBoundaryThreads, 1, 1);
-      lc.dynamicSmemBytes = smem;
-      lc.attrs = attr;
-      lc.numAttrs = 1;
-      int nclusters = 0;
-      e = cudaOccupancyMaxActiveClusters(&nclusters, fn, &lc);
-      if (e != cudaSuccess || nclusters <= 0) { cudaGetLastError(); continue; }
-      out->T = T; out->R = R; out->cluster = C; out->Dc = Dc;
-      out->smem = smem; out->max_clusters = nclusters; out->fn = fn;
+      const int n = max_active_clusters(fn, C, smem, kBoundaryThreads);
+      if (n <= 0) continue;
+      out->rf = false; out->T = T; out->R = R; out->cluster = C; out->Dc = Dc;
+      out->smem = smem; out->max_clusters = n; out->fn = fn;
       return ok();
     }
   }
@@ -191,18 +243,33 @@ respin_status_t respin_plan_create(respin_plan_t* out, int D, int r, const float
   if (r > 0) {
     respin_status_t st = configure_boundary(D, r_pad, (flags & RESPIN_H_FP32_DEBUG) != 0, &p->cfg);
     if (st != RESPIN_OK) { delete p; return st; }
-    // Factors as bf16 (round to nearest even): U^T [r_pad, D] then V [D, r_pad].
-    std::vector<__nv_bfloat16> host(static_cast<size_t>(2) * r_pad * D, __float2bfloat16_rn(0.f));
-    __nv_bfloat16* ut = host.data();
-    __nv_bfloat16* v = host.data() + static_cast<size_t>(r_pad) * D;
+    // Factors as bf16 (round to nearest even), zero padded to r_pad columns.
+    std::vector<uint16_t> ub(static_cast<size_t>(D) * r_pad, 0), vb(static_cast<size_t>(D) * r_pad, 0);
     for (int d = 0; d < D; ++d)
       for (int j = 0; j < r; ++j) {
-        ut[static_cast<size_t>(j) * D + d] = __float2bfloat16_rn(U_r[static_cast<size_t>(d) * r + j]);
-        v[static_cast<size_t>(d) * r_pad + j] = __float2bfloat16_rn(V_r[static_cast<size_t>(d) * r + j]);
+        const __nv_bfloat16 u = __float2bfloat16_rn(U_r[static_cast<size_t>(d) * r + j]);
+        const __nv_bfloat16 v = __float2bfloat16_rn(V_r[static_cast<size_t>(d) * r + j]);
+        ub[static_cast<size_t>(d) * r_pad + j] = *reinterpret_cast<const uint16_t*>(&u);
+        vb[static_cast<size_t>(d) * r_pad + j] = *reinterpret_cast<const uint16_t*>(&v);
       }
-    e = cudaMalloc(&p->factors, host.size() * sizeof(__nv_bfloat16));
+    // Device layout: fragment order for the register-factor kernel, else
+    // U^T [r_pad, D] followed by V [D, r_pad].
+    std::vector<uint32_t> dev_words(static_cast<size_t>(D) * r_pad, 0);  // 2 * D * r_pad bf16
+    if (p->cfg.rf) {
+      const size_t half = static_cast<size_t>(D) * r_pad / 2;
+      rf_pack_factors(ub.data(), vb.data(), D, r_pad, p->cfg.T, p->cfg.Dc, dev_words.data(), dev_words.data() + half);
+    } else {
+      uint16_t* h16 = reinterpret_cast<uint16_t*>(dev_words.data());
+      for (int d = 0; d < D; ++d)
+        for (int j = 0; j < r_pad; ++j) {
+          h16[static_cast<size_t>(j) * D + d] = ub[static_cast<size_t>(d) * r_pad + j];
+          h16[static_cast<size_t>(r_pad) * D + static_cast<size_t>(d) * r_pad + j] =
+              vb[static_cast<size_t>(d) * r_pad + j];
+        }
+    }
+    e = cudaMalloc(&p->factors, dev_words.size() * sizeof(uint32_t));
     if (e != cudaSuccess) { delete p; cudaGetLastError(); return fail(RESPIN_ERR_OOM, "cudaMalloc factors: %s", cudaGetErrorString(e)); }
-    e = cudaMemcpy(p->factors, host.data(), host.size() * sizeof(__nv_bfloat16), cudaMemcpyHostToDevice);
+    e = cudaMemcpy(p->factors, dev_words.data(), dev_words.size() * sizeof(uint32_t), cudaMemcpyHostToDevice);
     if (e != cudaSuccess) { cudaFree(p->factors); delete p; return cuda_fail(e, "cudaMemcpy factors"); }
   }
   // The row kernels need the shared-memory carve-out only for their reduction.
@@ -283,16 +350,24 @@ respin_status_t respin_boundary_forward(respin_plan_t plan, const void* x, const
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   lc.gridDim = dim3(nclusters * c.cluster, 1, 1);
-  lc.blockDim = dim3(kBoundaryThreads, 1, 1);
+  lc.blockDim = dim3(c.rf ? kRfThreads : kBoundaryThreads, 1, 1);
   lc.dynamicSmemBytes = c.smem;
   lc.stream = s;
   lc.attrs = attr;
   lc.numAttrs = 1;
-  const bf16* ut = plan->factors;
-  const bf16* v = plan->factors + static_cast<size_t>(plan->r_pad) * D;
-  int Dc = c.Dc;
-  void* args[] = {&xb, &rb, &ut, &v, &N, const_cast<int*>(&D), &Dc, &h_out, &q_packed, &scale};
-  cudaError_t e = cudaLaunchKernelExC(&lc, c.fn, args);
+  cudaError_t e;
+  if (c.rf) {
+    const uint4* uf = reinterpret_cast<const uint4*>(plan->factors);
+    const uint4* vf = reinterpret_cast<const uint4*>(plan->factors + static_cast<size_t>(plan->r_pad) * D);
+    void* args[] = {&xb, &rb, &uf, &vf, &N, const_cast<int*>(&D), &h_out, &q_packed, &scale};
+    e = cudaLaunchKernelExC(&lc, c.fn, args);
+  } else {
+    const bf16* ut = plan->factors;
+    const bf16* v = plan->factors + static_cast<size_t>(plan->r_pad) * D;
+    int Dc = c.Dc;
+    void* args[] = {&xb, &rb, &ut, &v, &N, const_cast<int*>(&D), &Dc, &h_out, &q_packed, &scale};
+    e = cudaLaunchKernelExC(&lc, c.fn, args);
+  }
   if (e != cudaSuccess) return cuda_fail(e, "boundary_cluster_kernel launch");
   return ok();
 }
@@ -314,6 +389,42 @@ static cudaError_t gemm_prepare(int dev) {
   return e;
 }
 
+// cuTensorMapEncodeTiled, fetched once through the runtime's driver entry
+// point (no link-time dependency on the driver library).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_tiled() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+    cudaGetLastError();
+  });
+  return fn;
+}
+
+// 2-D uint8 tensor map over a row-major [rows, cols] byte matrix with a box
+// of [box_rows, box_cols] (no swizzle, out-of-range reads return zeros).
+static bool make_tmap_u8(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols,
+                         uint32_t box_rows, uint32_t box_cols) {
+  EncodeTiledFn fn = encode_tiled();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 static respin_status_t gemm_common(const uint8_t* q_act, const float* scale_act, const uint8_t* q_w,
                                    const float* scale_w, int N, int K, int O, void* out,
                                    void* stream, bool i32) {
@@ -327,10 +438,8 @@ static respin_status_t gemm_common(const uint8_t* q_act, const float* scale_act,
     return fail(RESPIN_ERR_INVALID_ARG, "a required pointer is NULL");
   if (!aligned(q_act, 16) || !aligned(q_w, 16) || !aligned(out, 16))
     return fail(RESPIN_ERR_ALIGNMENT, "q_act, q_w and out must be 16-byte aligned");
-  if (!aligned(scale_act, 4) || !aligned(scale_w, 4))
-    return fail(RESPIN_ERR_ALIGNMENT, "scales must be 4-byte aligned");
-  if (static_cast<long long>((N + kGemmBM - 1) / kGemmBM) > 65535)
-    return fail(RESPIN_ERR_UNSUPPORTED, "N=%d too large", N);
+  if (!aligned(scale_act, 4) || !aligned(scale_w, 16))
+    return fail(RESPIN_ERR_ALIGNMENT, "scale_act must be 4-byte and scale_w 16-byte aligned");
   if (fault_at("launch")) return fail(RESPIN_ERR_CUDA, "injected fault at launch");
 
   int dev = 0;
@@ -338,12 +447,19 @@ static respin_status_t gemm_common(const uint8_t* q_act, const float* scale_act,
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
   e = gemm_prepare(dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gemm smem)");
-  dim3 grid((O + kGemmBN - 1) / kGemmBN, (N + kGemmBM - 1) / kGemmBM, 1);
+  int sms = 148;
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const long long tiles = static_cast<long long>((O + kGemmBN - 1) / kGemmBN) * ((N + kGemmBM - 1) / kGemmBM);
+  dim3 grid(static_cast<unsigned>(tiles < sms ? tiles : sms), 1, 1);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  CUtensorMap tmA, tmB;
+  if (!make_tmap_u8(&tmA, q_act, N, K / 2, kGemmBM, kGemmBK / 2) ||
+      !make_tmap_u8(&tmB, q_w, O, K / 2, kGemmBN, kGemmBK / 2))
+    return fail(RESPIN_ERR_CUDA, "cuTensorMapEncodeTiled failed for the GEMM operands");
   if (i32)
-    w4a4_gemm_kernel<true><<<grid, kGemmThreads, kGemmSmemBytes, s>>>(q_act, scale_act, q_w, scale_w, N, K, O, out);
+    w4a4_gemm_kernel<true><<<grid, kGemmThreads, kGemmSmemBytes, s>>>(tmA, tmB, scale_act, scale_w, N, K, O, out);
   else
-    w4a4_gemm_kernel<false><<<grid, kGemmThreads, kGemmSmemBytes, s>>>(q_act, scale_act, q_w, scale_w, N, K, O, out);
+    w4a4_gemm_kernel<false><<<grid, kGemmThreads, kGemmSmemBytes, s>>>(tmA, tmB, scale_act, scale_w, N, K, O, out);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "w4a4_gemm_kernel launch");
   return ok();

@@ -42,7 +42,7 @@ def run(qa, qw, sa, sw):
 def check(qa, qw, sa, sw, acc, outb, rows=None):
     if rows is not None:
         qa, sa, acc, outb = qa[rows], sa[rows], acc[rows], outb[rows]
-    ref = O.w4a4_acc(qa, qw)
+    ref = O.w4a4_acc_fp64(qa, qw)
     assert np.array_equal(acc.astype(np.int64), ref), "int32 accumulators differ"
     want = O.w4a4_epilogue_bits(ref, sa, sw)
     assert np.array_equal(outb, want), "bf16 outputs differ"
@@ -72,11 +72,20 @@ def test_gemm_decode_4096(N):
     check(qa, qw, sa, sw, acc, outb)
 
 
-def test_gemm_full_size_llama2_7b_sampled():
-    """2048 x 4096 -> 11008 (bench launch configuration), 64 sampled rows."""
+def test_gemm_full_size_llama2_7b():
+    """2048 x 4096 -> 11008 (bench launch configuration; several tiles per
+    persistent CTA), every output checked, twice in a row."""
     qa, qw, sa, sw = make(2048, 4096, 11008)
+    for _ in range(2):
+        acc, outb = run(qa, qw, sa, sw)
+        check(qa, qw, sa, sw, acc, outb)
+
+
+def test_gemm_full_size_llama3_8b_down_sampled():
+    """4096 x 14336 -> 4096 (down projection of the stack workload), 128 rows."""
+    qa, qw, sa, sw = make(4096, 14336, 4096, seed=2)
     acc, outb = run(qa, qw, sa, sw)
-    rows = np.sort(np.random.default_rng(3).choice(2048, 64, replace=False))
+    rows = np.sort(np.random.default_rng(4).choice(4096, 128, replace=False))
     check(qa, qw, sa, sw, acc, outb, rows)
 
 

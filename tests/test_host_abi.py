@@ -105,6 +105,7 @@ def gemm(qa=A16, sa=A16, qw=A16B, sw=A16B, N=4, K=256, O=32, out=A16):
     (dict(qa=MIS), rq.RESPIN_ERR_ALIGNMENT),
     (dict(out=MIS), rq.RESPIN_ERR_ALIGNMENT),
     (dict(sa=A16 + 2), rq.RESPIN_ERR_ALIGNMENT),
+    (dict(sw=A16B + 4), rq.RESPIN_ERR_ALIGNMENT),
 ])
 def test_gemm_validation(kw, want):
     assert gemm(**kw) == want

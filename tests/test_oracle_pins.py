@@ -286,6 +286,15 @@ def test_gemm_naive_loops():
     assert O.w4a4_acc(a, w).tolist() == ref
 
 
+def test_gemm_fp64_form_matches_integer_definition():
+    rs = np.random.default_rng(16)
+    a = rs.integers(0, 256, (37, 256), dtype=np.uint8)
+    w = rs.integers(0, 256, (29, 256), dtype=np.uint8)
+    assert np.array_equal(O.w4a4_acc_fp64(a, w), O.w4a4_acc(a, w))
+    ext_a = np.full((3, 64), 0x88, np.uint8)   # all -8: |acc| = 64 K
+    assert np.all(O.w4a4_acc_fp64(ext_a, ext_a) == 64 * 128)
+
+
 def test_gemm_selection_matrix():
     # One +1 per weight row selects one activation code: a gather.
     rs = np.random.default_rng(14)
