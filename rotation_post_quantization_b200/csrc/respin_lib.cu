@@ -372,21 +372,55 @@ respin_status_t respin_boundary_forward(respin_plan_t plan, const void* x, const
   return ok();
 }
 
+extern "C++" {
+template <int CG, bool I32>
+const void* gemm_fn() {
+  return reinterpret_cast<const void*>(&w4a4_gemm_kernel<CG, I32>);
+}
+}
+
 // The GEMM kernels need the large dynamic shared-memory carve-out; set it
-// once per device.
-static cudaError_t gemm_prepare(int dev) {
+// once per device and record how many CTA pairs can be co-resident.
+struct GemmDeviceInfo {
+  bool ready = false;
+  int sms = 0;
+  int max_pairs = 0;
+};
+
+static cudaError_t gemm_prepare(int dev, GemmDeviceInfo* info) {
   static std::mutex mu;
-  static bool done[256] = {};
+  static GemmDeviceInfo infos[256];
   if (dev < 0 || dev >= 256) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lk(mu);
-  if (done[dev]) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(&w4a4_gemm_kernel<false>),
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmemBytes);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(reinterpret_cast<const void*>(&w4a4_gemm_kernel<true>),
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmemBytes);
-  if (e == cudaSuccess) done[dev] = true;
-  return e;
+  GemmDeviceInfo& d = infos[dev];
+  if (!d.ready) {
+    cudaError_t e = cudaSuccess;
+    const void* fns[4] = {gemm_fn<1, false>(), gemm_fn<1, true>(), gemm_fn<2, false>(), gemm_fn<2, true>()};
+    const int smem[4] = {GemmCfg<1>::Smem, GemmCfg<1>::Smem, GemmCfg<2>::Smem, GemmCfg<2>::Smem};
+    for (int i = 0; i < 4 && e == cudaSuccess; ++i)
+      e = cudaFuncSetAttribute(fns[i], cudaFuncAttributeMaxDynamicSharedMemorySize, smem[i]);
+    if (e != cudaSuccess) return e;
+    e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t lc = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    lc.gridDim = dim3(2, 1, 1);
+    lc.blockDim = dim3(kGemmThreads, 1, 1);
+    lc.dynamicSmemBytes = GemmCfg<2>::Smem;
+    lc.attrs = attr;
+    lc.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(&d.max_pairs, fns[2], &lc) != cudaSuccess) {
+      cudaGetLastError();
+      d.max_pairs = 0;
+    }
+    d.ready = true;
+  }
+  *info = d;
+  return cudaSuccess;
 }
 
 // cuTensorMapEncodeTiled, fetched once through the runtime's driver entry
@@ -445,21 +479,40 @@ static respin_status_t gemm_common(const uint8_t* q_act, const float* scale_act,
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
-  e = gemm_prepare(dev);
+  GemmDeviceInfo info;
+  e = gemm_prepare(dev, &info);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gemm smem)");
-  int sms = 148;
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const long long tiles = static_cast<long long>((O + kGemmBN - 1) / kGemmBN) * ((N + kGemmBM - 1) / kGemmBM);
-  dim3 grid(static_cast<unsigned>(tiles < sms ? tiles : sms), 1, 1);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // CTA pairs (256-token tiles) from this many tokens on.
+#ifndef RESPIN_GEMM_PAIR_MIN_TOKENS
+#define RESPIN_GEMM_PAIR_MIN_TOKENS (1 << 30)
+#endif
+  const int CG = (N >= RESPIN_GEMM_PAIR_MIN_TOKENS && info.max_pairs > 0) ? 2 : 1;
+  const long long tiles = static_cast<long long>((O + kGemmBN - 1) / kGemmBN) *
+                          ((N + kGemmBM * CG - 1) / (kGemmBM * CG));
   CUtensorMap tmA, tmB;
   if (!make_tmap_u8(&tmA, q_act, N, K / 2, kGemmBM, kGemmBK / 2) ||
-      !make_tmap_u8(&tmB, q_w, O, K / 2, kGemmBN, kGemmBK / 2))
+      !make_tmap_u8(&tmB, q_w, O, K / 2, kGemmBN / CG, kGemmBK / 2))
     return fail(RESPIN_ERR_CUDA, "cuTensorMapEncodeTiled failed for the GEMM operands");
-  if (i32)
-    w4a4_gemm_kernel<true><<<grid, kGemmThreads, kGemmSmemBytes, s>>>(tmA, tmB, scale_act, scale_w, N, K, O, out);
-  else
-    w4a4_gemm_kernel<false><<<grid, kGemmThreads, kGemmSmemBytes, s>>>(tmA, tmB, scale_act, scale_w, N, K, O, out);
+  const void* fn = CG == 2 ? (i32 ? gemm_fn<2, true>() : gemm_fn<2, false>())
+                           : (i32 ? gemm_fn<1, true>() : gemm_fn<1, false>());
+  const long long groups = CG == 2 ? (tiles < info.max_pairs ? tiles : info.max_pairs)
+                                   : (tiles < info.sms ? tiles : info.sms);
+  cudaLaunchConfig_t lc = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CG;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  lc.gridDim = dim3(static_cast<unsigned>(groups * CG), 1, 1);
+  lc.blockDim = dim3(kGemmThreads, 1, 1);
+  lc.dynamicSmemBytes = CG == 2 ? GemmCfg<2>::Smem : GemmCfg<1>::Smem;
+  lc.stream = s;
+  lc.attrs = attr;
+  lc.numAttrs = 1;
+  void* args[] = {&tmA, &tmB, const_cast<float**>(&scale_act), const_cast<float**>(&scale_w), &N, &K, &O, &out};
+  e = cudaLaunchKernelExC(&lc, fn, args);
+  if (e != cudaSuccess) return cuda_fail(e, "w4a4_gemm_kernel launch");
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "w4a4_gemm_kernel launch");
   return ok();

@@ -20,19 +20,23 @@
 //    permutation, so the dot product over K is unchanged and no byte
 //    interleaving is needed.
 //
-// Structure (persistent, warp-specialised, one CTA per SM):
-//  * 1 TMA warp brings each packed K block (A: 128 rows x 64 bytes, B: 256 rows
-//    x 64 bytes) into a 3-stage packed ring with two 2-D tensor copies (rows
-//    past N or O arrive as zeros). Loading through TMA keeps the packed bytes
-//    off the LSU data pipe, where sector-granular global loads cost 4x the
-//    wavefronts of the shared-memory reads that replace them;
+// Structure (persistent, warp-specialised, one CTA per SM; CG = 1, or a pair
+// of CTAs with CG = 2):
+//  * 1 TMA warp brings each packed K block (this CTA's 128 token rows and its
+//    share of the channel rows, 64 bytes each) into a packed ring with two 2-D
+//    tensor copies (rows past N or O arrive as zeros). Loading through TMA
+//    keeps the packed bytes off the LSU data pipe, where sector-granular
+//    global loads cost 4x the wavefronts of the shared-memory reads that
+//    replace them;
 //  * 8 producer warps read the packed chunks (conflict-free 16-byte loads),
-//    widen them and store them into a 3-stage shared-memory ring in the
-//    128-byte-swizzled K-major canonical layout (128 tokens x 256 channels x
-//    128 K per stage, 48 KB);
-//  * 1 MMA warp: one thread issues 4 MMAs (M=128, N=256, K=32) per stage and
-//    commits to the stage's empty barrier; accumulators alternate between two
-//    256-column TMEM buffers;
+//    widen them and store them into a ring in the 128-byte-swizzled K-major
+//    canonical layout;
+//  * 1 MMA warp: one thread issues 4 MMAs (K = 32 each) per stage; the
+//    accumulators alternate between two 256-column TMEM buffers.
+//    CG = 1: M = 128, N = 256 per CTA. CG = 2: the leader CTA of the pair
+//    issues M = 256, N = 256 MMAs that read A rows and B channels from both
+//    CTAs (each CTA stages 128 token rows and 128 of the 256 channels), so
+//    every SM widens and stores half the weight bytes it would alone;
 //  * 4 epilogue warps drain the other TMEM buffer (tcgen05.ld), apply the two
 //    scales and store bf16, overlapping the next tile's main loop.
 #pragma once
@@ -45,100 +49,131 @@
 
 namespace respin {
 
-constexpr int kGemmBM = 128;
-constexpr int kGemmBN = 256;
 constexpr int kGemmBK = 128;                 // int8 K per stage (64 packed bytes per row)
-constexpr int kGemmStages = 3;               // widened (int8) stages
-constexpr int kGemmPStages = 3;              // packed (int4) stages
+constexpr int kGemmBM = 128;                 // token rows per CTA
+constexpr int kGemmBN = 256;                 // channels per tile
 constexpr int kGemmProducerWarps = 8;
 constexpr int kGemmEpilogueWarps = 4;
 constexpr int kGemmMmaWarp = kGemmProducerWarps;                 // warp 8
 constexpr int kGemmEpiWarp0 = kGemmProducerWarps + 1;            // warps 9..12
 constexpr int kGemmTmaWarp = kGemmEpiWarp0 + kGemmEpilogueWarps;  // warp 13
 constexpr int kGemmThreads = (kGemmTmaWarp + 1) * 32;
-constexpr int kGemmAStage = kGemmBM * kGemmBK;  // 16 KB
-constexpr int kGemmBStage = kGemmBN * kGemmBK;  // 32 KB
-constexpr int kGemmStageBytes = kGemmAStage + kGemmBStage;
-constexpr int kGemmPAStage = kGemmBM * kGemmBK / 2;   // 8 KB packed A
-constexpr int kGemmPStageBytes = (kGemmBM + kGemmBN) * kGemmBK / 2;  // 24 KB
-constexpr int kGemmChunks = (kGemmBM + kGemmBN) * (kGemmBK / 32);  // 16-byte packed chunks
-constexpr int kGemmChunksPerThread = kGemmChunks / (kGemmProducerWarps * 32);
-constexpr int kGemmSmemBytes =
-    kGemmStages * kGemmStageBytes + kGemmPStages * kGemmPStageBytes + 1024 + 256;
-static_assert(kGemmChunks % (kGemmProducerWarps * 32) == 0, "chunk split");
 
-// tmA: uint8 [N, K/2] box {64, 128}; tmB: uint8 [O, K/2] box {64, 256}
+#ifndef RESPIN_GEMM_US1
+#define RESPIN_GEMM_US1 3
+#endif
+#ifndef RESPIN_GEMM_PS1
+#define RESPIN_GEMM_PS1 3
+#endif
+#ifndef RESPIN_GEMM_US2
+#define RESPIN_GEMM_US2 4
+#endif
+#ifndef RESPIN_GEMM_PS2
+#define RESPIN_GEMM_PS2 4
+#endif
+
+template <int CG>
+struct GemmCfg {
+  static constexpr int BNC = kGemmBN / CG;              // channel rows staged by this CTA
+  static constexpr int US = CG == 1 ? RESPIN_GEMM_US1 : RESPIN_GEMM_US2;  // widened stages
+  static constexpr int PS = CG == 1 ? RESPIN_GEMM_PS1 : RESPIN_GEMM_PS2;  // packed stages
+  static constexpr int AStage = kGemmBM * kGemmBK;      // widened A bytes
+  static constexpr int BStage = BNC * kGemmBK;          // widened B bytes
+  static constexpr int Stage = AStage + BStage;
+  static constexpr int PAStage = kGemmBM * kGemmBK / 2; // packed A bytes
+  static constexpr int PStage = (kGemmBM + BNC) * kGemmBK / 2;
+  static constexpr int Chunks = (kGemmBM + BNC) * (kGemmBK / 32);  // 16-byte packed chunks
+  static constexpr int ChunksPerThread = Chunks / (kGemmProducerWarps * 32);
+  static constexpr int TileM = kGemmBM * CG;            // token rows per tile
+  static constexpr int Smem = US * Stage + PS * PStage + 1024 + 256;
+  static_assert(Chunks % (kGemmProducerWarps * 32) == 0, "chunk split");
+};
+
+// tmA: uint8 [N, K/2] box {64, 128}; tmB: uint8 [O, K/2] box {64, 256/CG}
 // (inner dimension first), no swizzle, out-of-range elements zero filled.
-template <bool I32OUT>
+template <int CG, bool I32OUT>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const float* __restrict__ sa, const float* __restrict__ sw, int N, int K,
                  int O, void* __restrict__ out) {
+  using G = GemmCfg<CG>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* smem = smem_raw + (base - raw);
-  const uint32_t pbase = base + kGemmStages * kGemmStageBytes;   // packed ring
-  const uint32_t bars = pbase + kGemmPStages * kGemmPStageBytes;
-  const uint32_t full0 = bars, empty0 = bars + 8 * kGemmStages;
-  const uint32_t pfull0 = bars + 16 * kGemmStages;
-  const uint32_t pempty0 = pfull0 + 8 * kGemmPStages;
-  const uint32_t afull0 = pempty0 + 8 * kGemmPStages;     // accumulator buffer b full: afull0 + 8b
-  const uint32_t aempty0 = afull0 + 16;                    // accumulator buffer b drained
+  const uint32_t pbase = base + G::US * G::Stage;   // packed ring
+  const uint32_t bars = pbase + G::PS * G::PStage;
+  const uint32_t full0 = bars;                       // [US] widened stage ready (leader counts both CTAs)
+  const uint32_t empty0 = full0 + 8 * G::US;         // [US] widened stage consumed (MMA commit)
+  const uint32_t pfull0 = empty0 + 8 * G::US;        // [PS] packed stage landed (TMA)
+  const uint32_t pempty0 = pfull0 + 8 * G::PS;       // [PS] packed stage consumed
+  const uint32_t afull0 = pempty0 + 8 * G::PS;       // [2] accumulator buffer full (MMA commit)
+  const uint32_t aempty0 = afull0 + 16;              // [2] accumulator buffer drained (leader)
   const uint32_t tslot = aempty0 + 16;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t rank = CG == 2 ? cluster_ctarank() : 0u;
+  const int group = CG == 2 ? static_cast<int>(blockIdx.x) / 2 : static_cast<int>(blockIdx.x);
+  const int ngroups = CG == 2 ? static_cast<int>(gridDim.x) / 2 : static_cast<int>(gridDim.x);
   const int KB = K / kGemmBK;
-  const int mtiles = (N + kGemmBM - 1) / kGemmBM;
+  const int mtiles = (N + G::TileM - 1) / G::TileM;
   const int ntiles = (O + kGemmBN - 1) / kGemmBN;
   const int tiles = mtiles * ntiles;
 
   if (tid == 0) {
-    for (int s = 0; s < kGemmStages; ++s) {
-      mbar_init(full0 + 8 * s, kGemmProducerWarps * 32);
+    for (int s = 0; s < G::US; ++s) {
+      mbar_init(full0 + 8 * s, CG * kGemmProducerWarps);
       mbar_init(empty0 + 8 * s, 1);
     }
-    for (int s = 0; s < kGemmPStages; ++s) {
+    for (int s = 0; s < G::PS; ++s) {
       mbar_init(pfull0 + 8 * s, 1);
-      mbar_init(pempty0 + 8 * s, kGemmProducerWarps * 32);
+      mbar_init(pempty0 + 8 * s, kGemmProducerWarps);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(afull0 + 8 * b, 1);
-      mbar_init(aempty0 + 8 * b, kGemmEpilogueWarps * 32);
+      mbar_init(aempty0 + 8 * b, CG * kGemmEpilogueWarps);
     }
     fence_mbarrier_init();
   }
   if (warp == 0) {
-    tmem_alloc(tslot, 512);
-    tmem_relinquish();
+    if constexpr (CG == 2) {
+      tmem_alloc_pair(tslot, 512);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tslot, 512);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  if constexpr (CG == 2) cluster_sync(); else __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + (tslot - base));
+  // barriers signalled in the leader CTA by both CTAs of the pair
+  const uint32_t full_leader0 = CG == 2 ? map_to_rank(full0, 0) : full0;
+  const uint32_t aempty_leader0 = CG == 2 ? map_to_rank(aempty0, 0) : aempty0;
 
   if (warp < kGemmProducerWarps) {
     // ------------------------------------------------ producers: widen packed -> int8
     bool ok = true;
     int kstep = 0;  // running k-block counter over all tiles (selects the stages)
-    for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
+    for (int t = group; t < tiles; t += ngroups) {
       for (int kb = 0; kb < KB; ++kb, ++kstep) {
-        const int ps = kstep % kGemmPStages, s = kstep % kGemmStages;
-        if (ok) ok = mbar_wait(pfull0 + 8 * ps, (kstep / kGemmPStages) & 1, kSiteGemmPackedFull);
-        const uint8_t* pk = smem + (pbase - base) + ps * kGemmPStageBytes;
-        uint4 b[kGemmChunksPerThread];
+        const int ps = kstep % G::PS, s = kstep % G::US;
+        if (ok) ok = mbar_wait(pfull0 + 8 * ps, (kstep / G::PS) & 1, kSiteGemmPackedFull);
+        const uint8_t* pk = smem + (pbase - base) + ps * G::PStage;
+        uint4 b[G::ChunksPerThread];
 #pragma unroll
-        for (int j = 0; j < kGemmChunksPerThread; ++j)   // chunk q = row*4 + c, 16 bytes each
+        for (int j = 0; j < G::ChunksPerThread; ++j)   // chunk q = row*4 + c, 16 bytes each
           b[j] = *reinterpret_cast<const uint4*>(pk + (tid + j * kGemmProducerWarps * 32) * 16);
-        if (ok) ok = mbar_wait(empty0 + 8 * s, ((kstep / kGemmStages) & 1) ^ 1, kSiteGemmEmpty);
-        uint8_t* sA = smem + s * kGemmStageBytes;
+        if (ok) ok = mbar_wait(empty0 + 8 * s, ((kstep / G::US) & 1) ^ 1, kSiteGemmEmpty);
+        uint8_t* sA = smem + s * G::Stage;
 #pragma unroll
-        for (int j = 0; j < kGemmChunksPerThread; ++j) {
+        for (int j = 0; j < G::ChunksPerThread; ++j) {
           const int q = tid + j * kGemmProducerWarps * 32;
           const bool is_a = q < kGemmBM * 4;
           const int qq = is_a ? q : q - kGemmBM * 4;
           const int row = qq >> 2, c = qq & 3;
-          uint8_t* rowp = sA + (is_a ? 0 : kGemmAStage) + (row >> 3) * 1024 + (row & 7) * 128;
+          uint8_t* rowp = sA + (is_a ? 0 : G::AStage) + (row >> 3) * 1024 + (row & 7) * 128;
           const uint4 p = b[j];
           const uint4 lo = make_uint4((p.x << 4) & 0xF0F0F0F0u, (p.y << 4) & 0xF0F0F0F0u,
                                       (p.z << 4) & 0xF0F0F0F0u, (p.w << 4) & 0xF0F0F0F0u);
@@ -147,72 +182,86 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
           *reinterpret_cast<uint4*>(rowp + (((2 * c) ^ (row & 7)) << 4)) = lo;
           *reinterpret_cast<uint4*>(rowp + (((2 * c + 1) ^ (row & 7)) << 4)) = hi;
         }
-        // Widened stage -> MMA (async proxy reads): proxy fence, then signal.
+        // Widened stage -> MMA (async-proxy reads): every thread fences its
+        // own writes, then one lane per warp signals (release, cluster scope).
         // The packed stage is released only now, after its bytes were
         // consumed, so the next TMA refill (async-proxy write) cannot land
         // before these shared-memory reads retired.
         fence_proxy_async_smem();
-        mbar_arrive(full0 + 8 * s);
-        mbar_arrive(pempty0 + 8 * ps);
+        __syncwarp();
+        if (lane == 0) {
+          if constexpr (CG == 2) mbar_arrive_cluster(full_leader0 + 8 * s);
+          else mbar_arrive(full0 + 8 * s);
+          mbar_arrive(pempty0 + 8 * ps);
+        }
       }
     }
   } else if (warp == kGemmTmaWarp) {
     // ------------------------------------------------ TMA warp: packed K blocks
     bool ok = true;
     int kstep = 0;
-    for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
-      const int m0 = (t / ntiles) * kGemmBM, n0 = (t % ntiles) * kGemmBN;
+    for (int t = group; t < tiles; t += ngroups) {
+      const int arow = (t / ntiles) * G::TileM + static_cast<int>(rank) * kGemmBM;
+      const int brow = (t % ntiles) * kGemmBN + static_cast<int>(rank) * G::BNC;
       for (int kb = 0; kb < KB; ++kb, ++kstep) {
-        const int ps = kstep % kGemmPStages;
-        if (ok) ok = mbar_wait(pempty0 + 8 * ps, ((kstep / kGemmPStages) & 1) ^ 1, kSiteGemmPackedEmpty);
+        const int ps = kstep % G::PS;
+        if (ok) ok = mbar_wait(pempty0 + 8 * ps, ((kstep / G::PS) & 1) ^ 1, kSiteGemmPackedEmpty);
         if (lane == 0) {
-          const uint32_t dst = pbase + ps * kGemmPStageBytes;
-          mbar_arrive_expect_tx(pfull0 + 8 * ps, kGemmPStageBytes);
-          tma_load_2d(dst, &tmA, kb * (kGemmBK / 2), m0, pfull0 + 8 * ps);
-          tma_load_2d(dst + kGemmPAStage, &tmB, kb * (kGemmBK / 2), n0, pfull0 + 8 * ps);
+          const uint32_t dst = pbase + ps * G::PStage;
+          mbar_arrive_expect_tx(pfull0 + 8 * ps, G::PStage);
+          tma_load_2d(dst, &tmA, kb * (kGemmBK / 2), arow, pfull0 + 8 * ps);
+          tma_load_2d(dst + G::PAStage, &tmB, kb * (kGemmBK / 2), brow, pfull0 + 8 * ps);
         }
         __syncwarp();
       }
     }
   } else if (warp == kGemmMmaWarp) {
-    // ------------------------------------------------ MMA issuer (one warp)
-    constexpr uint32_t idesc = umma_idesc_s8(kGemmBM, kGemmBN);
-    bool ok = true;
-    int kstep = 0, local = 0;
-    for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++local) {
-      const int ab = local & 1;
-      // wait until the epilogue drained this accumulator buffer (two tiles ago)
-      if (ok) ok = mbar_wait(aempty0 + 8 * ab, ((local >> 1) & 1) ^ 1, kSiteGemmAccum);
-      tc_fence_after();
-      const uint32_t dtm = tmem + ab * kGemmBN;
-      for (int kb = 0; kb < KB; ++kb, ++kstep) {
-        const int s = kstep % kGemmStages;
-        if (ok) ok = mbar_wait(full0 + 8 * s, (kstep / kGemmStages) & 1, kSiteGemmFull);
+    // ------------------------------------------------ MMA issuer (leader CTA)
+    if (CG == 1 || rank == 0) {
+      constexpr uint32_t idesc = umma_idesc_s8(kGemmBM * CG, kGemmBN);
+      bool ok = true;
+      int kstep = 0, local = 0;
+      for (int t = group; t < tiles; t += ngroups, ++local) {
+        const int ab = local & 1;
+        // wait until both epilogues drained this accumulator buffer (two tiles ago)
+        if (ok) ok = mbar_wait_cluster(aempty0 + 8 * ab, ((local >> 1) & 1) ^ 1, kSiteGemmAccum);
         tc_fence_after();
-        if (lane == 0 && ok) {
-          const uint32_t a_addr = base + s * kGemmStageBytes;
-          const uint32_t b_addr = a_addr + kGemmAStage;
+        const uint32_t dtm = tmem + ab * kGemmBN;
+        for (int kb = 0; kb < KB; ++kb, ++kstep) {
+          const int s = kstep % G::US;
+          if (ok) ok = mbar_wait_cluster(full0 + 8 * s, (kstep / G::US) & 1, kSiteGemmFull);
+          tc_fence_after();
+          if (lane == 0 && ok) {
+            const uint32_t a_addr = base + s * G::Stage;
+            const uint32_t b_addr = a_addr + G::AStage;
 #pragma unroll
-          for (int k = 0; k < kGemmBK / 32; ++k)
-            tc_mma_i8(dtm, umma_desc_sw128(a_addr + 32 * k), umma_desc_sw128(b_addr + 32 * k), idesc,
-                      (kb | k) != 0 ? 1u : 0u);
-          tc_commit(empty0 + 8 * s);
+            for (int k = 0; k < kGemmBK / 32; ++k) {
+              const uint64_t ad = umma_desc_sw128(a_addr + 32 * k), bd = umma_desc_sw128(b_addr + 32 * k);
+              const uint32_t acc = (kb | k) != 0 ? 1u : 0u;
+              if constexpr (CG == 2) tc_mma_i8_pair(dtm, ad, bd, idesc, acc);
+              else tc_mma_i8(dtm, ad, bd, idesc, acc);
+            }
+            if constexpr (CG == 2) tc_commit_pair_multicast(empty0 + 8 * s, 0x3);
+            else tc_commit(empty0 + 8 * s);
+          }
+          __syncwarp();
+        }
+        if (lane == 0) {
+          if constexpr (CG == 2) tc_commit_pair_multicast(afull0 + 8 * ab, 0x3);
+          else tc_commit(afull0 + 8 * ab);
         }
         __syncwarp();
       }
-      if (lane == 0) tc_commit(afull0 + 8 * ab);
-      __syncwarp();
     }
   } else {
     // ------------------------------------------------ epilogue warps
-    const int ew = warp - kGemmEpiWarp0;   // TMEM lane quadrant of this warp
-    const int quad = warp & 3;             // hardware rule: warp w reads lanes 32*(w%4)..
-    (void)ew;
+    const int quad = warp & 3;   // hardware rule: warp w reads TMEM lanes 32*(w%4)..
     bool ok = true;
     int local = 0;
-    for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++local) {
+    for (int t = group; t < tiles; t += ngroups, ++local) {
       const int ab = local & 1;
-      const int m0 = (t / ntiles) * kGemmBM, n0 = (t % ntiles) * kGemmBN;
+      const int m0 = (t / ntiles) * G::TileM + static_cast<int>(rank) * kGemmBM;
+      const int n0 = (t % ntiles) * kGemmBN;
       if (ok) ok = mbar_wait(afull0 + 8 * ab, (local >> 1) & 1, kSiteGemmAccum);
       tc_fence_after();
       const int row = m0 + quad * 32 + lane;
@@ -255,16 +304,23 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
           }
         }
       }
-      // hand the accumulator buffer back to the MMA warp
+      // hand the accumulator buffer back to the MMA warp (of the leader CTA)
       tc_fence_before();
-      mbar_arrive(aempty0 + 8 * ab);
+      __syncwarp();
+      if (lane == 0) {
+        if constexpr (CG == 2) mbar_arrive_cluster(aempty_leader0 + 8 * ab);
+        else mbar_arrive(aempty0 + 8 * ab);
+      }
     }
   }
   tc_fence_before();
-  __syncthreads();
+  // Neither CTA of a pair may release its TMEM or shared memory while the
+  // other can still reach it.
+  if constexpr (CG == 2) cluster_sync(); else __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    if constexpr (CG == 2) tmem_dealloc_pair(tmem, 512);
+    else tmem_dealloc(tmem, 512);
   }
 }
 
