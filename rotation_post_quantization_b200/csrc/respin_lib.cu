@@ -459,6 +459,21 @@ static bool make_tmap_u8(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_
             CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2-D tensor map over the GEMM output [rows, cols] (bf16 or int32) for the
+// epilogue's tensor stores: box of 64 bytes x 32 rows, 64-byte swizzle.
+static bool make_tmap_out(CUtensorMap* m, void* ptr, uint64_t rows, uint64_t cols, bool i32) {
+  EncodeTiledFn fn = encode_tiled();
+  if (!fn) return false;
+  const uint32_t es = i32 ? 4u : 2u;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * es};
+  const cuuint32_t box[2] = {64u / es, 32u};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, i32 ? CU_TENSOR_MAP_DATA_TYPE_INT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ptr, dims,
+            strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+            CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 static respin_status_t gemm_common(const uint8_t* q_act, const float* scale_act, const uint8_t* q_w,
                                    const float* scale_w, int N, int K, int O, void* out,
                                    void* stream, bool i32) {
@@ -485,15 +500,16 @@ static respin_status_t gemm_common(const uint8_t* q_act, const float* scale_act,
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   // CTA pairs (256-token tiles) from this many tokens on.
 #ifndef RESPIN_GEMM_PAIR_MIN_TOKENS
-#define RESPIN_GEMM_PAIR_MIN_TOKENS (1 << 30)
+#define RESPIN_GEMM_PAIR_MIN_TOKENS (kGemmBM + 1)
 #endif
   const int CG = (N >= RESPIN_GEMM_PAIR_MIN_TOKENS && info.max_pairs > 0) ? 2 : 1;
   const long long tiles = static_cast<long long>((O + kGemmBN - 1) / kGemmBN) *
                           ((N + kGemmBM * CG - 1) / (kGemmBM * CG));
-  CUtensorMap tmA, tmB;
+  CUtensorMap tmA, tmB, tmO;
   if (!make_tmap_u8(&tmA, q_act, N, K / 2, kGemmBM, kGemmBK / 2) ||
-      !make_tmap_u8(&tmB, q_w, O, K / 2, kGemmBN / CG, kGemmBK / 2))
-    return fail(RESPIN_ERR_CUDA, "cuTensorMapEncodeTiled failed for the GEMM operands");
+      !make_tmap_u8(&tmB, q_w, O, K / 2, kGemmBN / CG, kGemmBK / 2) ||
+      !make_tmap_out(&tmO, out, N, O, i32))
+    return fail(RESPIN_ERR_CUDA, "cuTensorMapEncodeTiled failed for the GEMM operands or output");
   const void* fn = CG == 2 ? (i32 ? gemm_fn<2, true>() : gemm_fn<2, false>())
                            : (i32 ? gemm_fn<1, true>() : gemm_fn<1, false>());
   const long long groups = CG == 2 ? (tiles < info.max_pairs ? tiles : info.max_pairs)
@@ -510,7 +526,7 @@ static respin_status_t gemm_common(const uint8_t* q_act, const float* scale_act,
   lc.stream = s;
   lc.attrs = attr;
   lc.numAttrs = 1;
-  void* args[] = {&tmA, &tmB, const_cast<float**>(&scale_act), const_cast<float**>(&scale_w), &N, &K, &O, &out};
+  void* args[] = {&tmA, &tmB, &tmO, const_cast<float**>(&scale_act), const_cast<float**>(&scale_w), &N, &K, &O};
   e = cudaLaunchKernelExC(&lc, fn, args);
   if (e != cudaSuccess) return cuda_fail(e, "w4a4_gemm_kernel launch");
   e = cudaGetLastError();

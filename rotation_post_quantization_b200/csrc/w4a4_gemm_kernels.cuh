@@ -63,7 +63,10 @@ constexpr int kGemmThreads = (kGemmTmaWarp + 1) * 32;
 #define RESPIN_GEMM_US1 3
 #endif
 #ifndef RESPIN_GEMM_PS1
-#define RESPIN_GEMM_PS1 3
+#define RESPIN_GEMM_PS1 2
+#endif
+#ifndef RESPIN_GEMM_EB
+#define RESPIN_GEMM_EB 2
 #endif
 #ifndef RESPIN_GEMM_US2
 #define RESPIN_GEMM_US2 4
@@ -85,24 +88,48 @@ struct GemmCfg {
   static constexpr int Chunks = (kGemmBM + BNC) * (kGemmBK / 32);  // 16-byte packed chunks
   static constexpr int ChunksPerThread = Chunks / (kGemmProducerWarps * 32);
   static constexpr int TileM = kGemmBM * CG;            // token rows per tile
-  static constexpr int Smem = US * Stage + PS * PStage + 1024 + 256;
+  static constexpr int EB = RESPIN_GEMM_EB;             // output staging units per epilogue warp
+  static constexpr int Unit = 32 * 64;                  // one unit: 32 rows x 64 bytes
+  static constexpr int SwBytes = kGemmBN * 4;          // one tile's channel scales, per epilogue warp
+  static constexpr int Smem =
+      US * Stage + PS * PStage + kGemmEpilogueWarps * (EB * Unit + SwBytes) + 1024 + 256;
   static_assert(Chunks % (kGemmProducerWarps * 32) == 0, "chunk split");
 };
 
+// Exact int32 -> binary32 for |a| <= 2^22: adding a to the bit pattern of
+// 1.5 * 2^23 gives the float 1.5 * 2^23 + a (the sum stays within
+// [2^23, 2^24], where consecutive floats are the integers), and subtracting
+// 1.5 * 2^23 is exact. Two full-rate ALU operations instead of a conversion.
+__device__ __forceinline__ float exact_i22_to_f32(int32_t a) {
+  return __int_as_float(a + 0x4B400000) - 12582912.0f;
+}
+
+// Byte offset of 16-byte piece j (0..3) of row r (0..31) in a 32 x 64-byte
+// staging unit in the tensor-map 64-byte swizzle (piece index XOR bits 7-8 of
+// the offset). The unit starts on a 1024-byte boundary. Rows written by the
+// eight lanes of one quarter-warp land in eight distinct bank groups.
+__device__ __forceinline__ uint32_t sw64_offset(int r, int j) {
+  return static_cast<uint32_t>(r * 64 + ((j ^ ((r >> 1) & 3)) << 4));
+}
+
 // tmA: uint8 [N, K/2] box {64, 128}; tmB: uint8 [O, K/2] box {64, 256/CG}
 // (inner dimension first), no swizzle, out-of-range elements zero filled.
+// tmO: the output [N, O] (bf16, or int32 for I32OUT), box {64 bytes, 32 rows},
+// 64-byte swizzle; the store clips rows >= N and columns >= O.
 template <int CG, bool I32OUT>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                 const float* __restrict__ sa, const float* __restrict__ sw, int N, int K,
-                 int O, void* __restrict__ out) {
+                 const __grid_constant__ CUtensorMap tmO, const float* __restrict__ sa,
+                 const float* __restrict__ sw, int N, int K, int O) {
   using G = GemmCfg<CG>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* smem = smem_raw + (base - raw);
   const uint32_t pbase = base + G::US * G::Stage;   // packed ring
-  const uint32_t bars = pbase + G::PS * G::PStage;
+  const uint32_t ebase = pbase + G::PS * G::PStage;  // output staging units
+  const uint32_t swbase = ebase + kGemmEpilogueWarps * G::EB * G::Unit;  // channel scales
+  const uint32_t bars = swbase + kGemmEpilogueWarps * G::SwBytes;
   const uint32_t full0 = bars;                       // [US] widened stage ready (leader counts both CTAs)
   const uint32_t empty0 = full0 + 8 * G::US;         // [US] widened stage consumed (MMA commit)
   const uint32_t pfull0 = empty0 + 8 * G::US;        // [PS] packed stage landed (TMA)
@@ -255,52 +282,108 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     }
   } else {
     // ------------------------------------------------ epilogue warps
+    // Each warp owns 32 accumulator rows (TMEM lanes) and EB staging units.
+    // Per 32-column chunk: tcgen05.ld (lane = row, registers = columns),
+    // scale, write the row's 64 bytes (bf16) into a swizzled unit, and one
+    // lane issues a TMA tensor store of the 32 x 32 block, so every output
+    // row segment reaches L2 as whole sectors. int32 output takes two units
+    // (16 columns each) per chunk.
     const int quad = warp & 3;   // hardware rule: warp w reads TMEM lanes 32*(w%4)..
+    const uint32_t ubase = ebase + static_cast<uint32_t>(quad * G::EB * G::Unit);
+    float* sws = reinterpret_cast<float*>(smem + (swbase - base) + quad * G::SwBytes);
     bool ok = true;
-    int local = 0;
+    int local = 0, unit = 0;
+    auto stage_unit = [&](const uint4 (&piece)[4], int x, int y) {
+      if (lane == 0) bulk_wait_group_read<G::EB - 1>();   // this unit's previous store read it
+      __syncwarp();
+      const uint32_t u = ubase + static_cast<uint32_t>((unit % G::EB) * G::Unit);
+      uint8_t* up = smem + (u - base);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) *reinterpret_cast<uint4*>(up + sw64_offset(lane, j)) = piece[j];
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_2d(&tmO, x, y, u);
+        bulk_commit_group();
+      }
+      ++unit;
+    };
     for (int t = group; t < tiles; t += ngroups, ++local) {
       const int ab = local & 1;
       const int m0 = (t / ntiles) * G::TileM + static_cast<int>(rank) * kGemmBM;
       const int n0 = (t % ntiles) * kGemmBN;
+      const int y = m0 + quad * 32;           // first row of this warp's blocks
+      const int row = y + lane;
+      // Fetch the tile's scales while its accumulators are still being
+      // computed: sa for this lane's row, 8 channel scales per lane.
+      float sa_r = 0.f;
+      float4 sw0 = make_float4(0.f, 0.f, 0.f, 0.f), sw1 = sw0;
+      if constexpr (!I32OUT) {
+        if (row < N) sa_r = __ldg(sa + row);
+        if (n0 + 8 * lane < O) {   // O % 16 == 0: then all 8 channels are in range
+          sw0 = __ldg(reinterpret_cast<const float4*>(sw + n0 + 8 * lane));
+          sw1 = __ldg(reinterpret_cast<const float4*>(sw + n0 + 8 * lane + 4));
+        }
+      }
       if (ok) ok = mbar_wait(afull0 + 8 * ab, (local >> 1) & 1, kSiteGemmAccum);
+      ok = __all_sync(0xffffffffu, ok);
       tc_fence_after();
-      const int row = m0 + quad * 32 + lane;
-      const float sa_r = (row < N && !I32OUT) ? __ldg(sa + row) : 0.f;
+      if constexpr (!I32OUT) {
+        reinterpret_cast<float4*>(sws)[2 * lane] = sw0;
+        reinterpret_cast<float4*>(sws)[2 * lane + 1] = sw1;
+        __syncwarp();
+      }
+      const uint32_t tbase = tmem + (static_cast<uint32_t>(quad * 32) << 16) + ab * kGemmBN;
 #pragma unroll 1
-      for (int cc = 0; cc < kGemmBN / 32; ++cc) {
-        const int colb = n0 + cc * 32;
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + ab * kGemmBN + cc * 32, v);
+      for (int cc = 0; cc < kGemmBN / 32; cc += 2) {
+        uint32_t v[2][32];
+        tmem_ld_32x32b_x32(tbase + cc * 32, v[0]);
+        tmem_ld_32x32b_x32(tbase + cc * 32 + 32, v[1]);
         tmem_wait_ld();
-        if (!ok || row >= N) continue;
-        if constexpr (I32OUT) {
-          int32_t* op = static_cast<int32_t*>(out) + static_cast<size_t>(row) * O + colb;
+        if (!ok || y >= N) continue;
 #pragma unroll
-          for (int e = 0; e < 32; e += 4) {
-            if (colb + e >= O) break;
-            *reinterpret_cast<int4*>(op + e) =
-                make_int4(static_cast<int32_t>(v[e]) >> 8, static_cast<int32_t>(v[e + 1]) >> 8,
-                          static_cast<int32_t>(v[e + 2]) >> 8, static_cast<int32_t>(v[e + 3]) >> 8);
-          }
-        } else {
-          __nv_bfloat16* op = static_cast<__nv_bfloat16*>(out) + static_cast<size_t>(row) * O + colb;
+        for (int h = 0; h < 2; ++h) {
+          const int colb = n0 + (cc + h) * 32;
+          if (colb >= O) break;
+          if constexpr (I32OUT) {
 #pragma unroll
-          for (int e = 0; e < 32; e += 8) {
-            if (colb + e >= O) break;
-            const float4 w0 = __ldg(reinterpret_cast<const float4*>(sw + colb + e));
-            const float4 w1 = __ldg(reinterpret_cast<const float4*>(sw + colb + e + 4));
-            const float ws[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-            uint32_t w[4];
+            for (int half = 0; half < 2; ++half) {
+              if (colb + 16 * half >= O) break;
+              uint4 piece[4];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const int e0 = e + 2 * u;
-              const float f0 = __fmul_rn(
-                  __fmul_rn(static_cast<float>(static_cast<int32_t>(v[e0]) >> 8), sa_r), ws[2 * u]);
-              const float f1 = __fmul_rn(
-                  __fmul_rn(static_cast<float>(static_cast<int32_t>(v[e0 + 1]) >> 8), sa_r), ws[2 * u + 1]);
-              w[u] = pack_bf16x2(f0, f1);
+              for (int j = 0; j < 4; ++j) {
+                const int e = 16 * half + 4 * j;
+                piece[j] = make_uint4(static_cast<uint32_t>(static_cast<int32_t>(v[h][e]) >> 8),
+                                      static_cast<uint32_t>(static_cast<int32_t>(v[h][e + 1]) >> 8),
+                                      static_cast<uint32_t>(static_cast<int32_t>(v[h][e + 2]) >> 8),
+                                      static_cast<uint32_t>(static_cast<int32_t>(v[h][e + 3]) >> 8));
+              }
+              stage_unit(piece, colb + 16 * half, y);
             }
-            *reinterpret_cast<uint4*>(op + e) = make_uint4(w[0], w[1], w[2], w[3]);
+          } else {
+            uint4 piece[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              if (colb + 8 * j >= O) {   // O % 16 == 0: a chunk is full or half full
+                piece[j] = make_uint4(0u, 0u, 0u, 0u);
+                continue;
+              }
+              const float4 w0 = reinterpret_cast<const float4*>(sws)[(colb - n0) / 4 + 2 * j];
+              const float4 w1 = reinterpret_cast<const float4*>(sws)[(colb - n0) / 4 + 2 * j + 1];
+              const float ws[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+              uint32_t w[4];
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                const int e = 8 * j + 2 * u;
+                const float f0 = __fmul_rn(
+                    __fmul_rn(exact_i22_to_f32(static_cast<int32_t>(v[h][e]) >> 8), sa_r), ws[2 * u]);
+                const float f1 = __fmul_rn(
+                    __fmul_rn(exact_i22_to_f32(static_cast<int32_t>(v[h][e + 1]) >> 8), sa_r), ws[2 * u + 1]);
+                w[u] = pack_bf16x2(f0, f1);
+              }
+              piece[j] = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+            stage_unit(piece, colb, y);
           }
         }
       }
@@ -312,6 +395,9 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         else mbar_arrive(aempty0 + 8 * ab);
       }
     }
+    // the staging units must not be released while a store still reads them
+    if (lane == 0) bulk_wait_group_all();
+    __syncwarp();
   }
   tc_fence_before();
   // Neither CTA of a pair may release its TMEM or shared memory while the
