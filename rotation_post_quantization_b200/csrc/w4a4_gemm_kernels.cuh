@@ -27,7 +27,13 @@
 //    tensor copies (rows past N or O arrive as zeros). Loading through TMA
 //    keeps the packed bytes off the LSU data pipe, where sector-granular
 //    global loads cost 4x the wavefronts of the shared-memory reads that
-//    replace them;
+//    replace them. Bulk copies issued by one thread complete one after the
+//    other (about 0.3 us each on B200, whatever their size), while copies
+//    from different threads overlap, so 2 * PS lanes issue: lane 2p + o
+//    copies operand o (A or B) of every K block that lands in packed stage
+//    p. One lane pair per stage keeps each stage's waits in order (a lane
+//    serving two stages could run two phases ahead of a barrier, where the
+//    parity test no longer tells the phases apart);
 //  * 8 producer warps read the packed chunks (conflict-free 16-byte loads),
 //    widen them and store them into a ring in the 128-byte-swizzled K-major
 //    canonical layout;
@@ -94,6 +100,7 @@ struct GemmCfg {
   static constexpr int Smem =
       US * Stage + PS * PStage + kGemmEpilogueWarps * (EB * Unit + SwBytes) + 1024 + 256;
   static_assert(Chunks % (kGemmProducerWarps * 32) == 0, "chunk split");
+  static_assert(2 * PS <= 32, "one issuing lane pair per packed stage");
 };
 
 // Exact int32 -> binary32 for |a| <= 2^22: adding a to the bit pattern of
@@ -153,7 +160,7 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       mbar_init(empty0 + 8 * s, 1);
     }
     for (int s = 0; s < G::PS; ++s) {
-      mbar_init(pfull0 + 8 * s, 1);
+      mbar_init(pfull0 + 8 * s, 2);   // the A and the B copy each arrive with their bytes
       mbar_init(pempty0 + 8 * s, kGemmProducerWarps);
     }
     for (int b = 0; b < 2; ++b) {
@@ -210,10 +217,11 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
           *reinterpret_cast<uint4*>(rowp + (((2 * c + 1) ^ (row & 7)) << 4)) = hi;
         }
         // Widened stage -> MMA (async-proxy reads): every thread fences its
-        // own writes, then one lane per warp signals (release, cluster scope).
-        // The packed stage is released only now, after its bytes were
-        // consumed, so the next TMA refill (async-proxy write) cannot land
-        // before these shared-memory reads retired.
+        // own writes, then one lane per warp signals. The packed stage is
+        // released only now: the same proxy fence orders the reads of its
+        // bytes (generic proxy) before the next tensor copy into it (async
+        // proxy). A separate fence right after the reads costs more than the
+        // earlier release gains.
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
@@ -225,21 +233,25 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     }
   } else if (warp == kGemmTmaWarp) {
     // ------------------------------------------------ TMA warp: packed K blocks
-    bool ok = true;
-    int kstep = 0;
-    for (int t = group; t < tiles; t += ngroups) {
-      const int arow = (t / ntiles) * G::TileM + static_cast<int>(rank) * kGemmBM;
-      const int brow = (t % ntiles) * kGemmBN + static_cast<int>(rank) * G::BNC;
-      for (int kb = 0; kb < KB; ++kb, ++kstep) {
-        const int ps = kstep % G::PS;
-        if (ok) ok = mbar_wait(pempty0 + 8 * ps, ((kstep / G::PS) & 1) ^ 1, kSiteGemmPackedEmpty);
-        if (lane == 0) {
+    if (lane < 2 * G::PS) {
+      const int stage = lane >> 1;
+      const bool is_b = (lane & 1) != 0;
+      const uint32_t bytes = is_b ? G::PStage - G::PAStage : G::PAStage;
+      bool ok = true;
+      int kstep = 0;
+      for (int t = group; t < tiles; t += ngroups) {
+        const int arow = (t / ntiles) * G::TileM + static_cast<int>(rank) * kGemmBM;
+        const int brow = (t % ntiles) * kGemmBN + static_cast<int>(rank) * G::BNC;
+        for (int kb = 0; kb < KB; ++kb, ++kstep) {
+          const int ps = kstep % G::PS;
+          if (ps != stage) continue;
+          if (ok) ok = mbar_wait(pempty0 + 8 * ps, ((kstep / G::PS) & 1) ^ 1, kSiteGemmPackedEmpty);
+          if (!ok) continue;
           const uint32_t dst = pbase + ps * G::PStage;
-          mbar_arrive_expect_tx(pfull0 + 8 * ps, G::PStage);
-          tma_load_2d(dst, &tmA, kb * (kGemmBK / 2), arow, pfull0 + 8 * ps);
-          tma_load_2d(dst + G::PAStage, &tmB, kb * (kGemmBK / 2), brow, pfull0 + 8 * ps);
+          mbar_arrive_expect_tx(pfull0 + 8 * ps, bytes);
+          if (is_b) tma_load_2d(dst + G::PAStage, &tmB, kb * (kGemmBK / 2), brow, pfull0 + 8 * ps);
+          else tma_load_2d(dst, &tmA, kb * (kGemmBK / 2), arow, pfull0 + 8 * ps);
         }
-        __syncwarp();
       }
     }
   } else if (warp == kGemmMmaWarp) {
