@@ -1,0 +1,344 @@
+// Row-tile block-boundary kernel: the rank-r basis fix and per-token INT4
+// quantization for 16 whole tokens per CTA (r <= 32, D = 1024 / 2048 / 4096).
+//
+// Same arithmetic as the cluster kernels (subspace residual rotation of the
+// ReSpinQuant explainers, zh §2.2 steps 1-3, row convention, then W4A4
+// activation quantization, zh §3-§4):
+//   y = residual U ;  h = (residual + x) + y V^T  (fp32) ;  h' = bf16(h)
+//   amax = max|h'| ; inv = 7/amax ; q = rint(h' inv)
+//
+// Design (one CTA per SM, persistent over 16-token tiles, no cluster):
+//  * the residual tile (16 x D bf16) is brought into shared memory by 2-D
+//    tensor copies of 64-column blocks (16 rows x 128 bytes, 128-byte
+//    swizzle: conflict-free ldmatrix and fragment accesses) and is turned into
+//    h' in place;
+//  * warp w owns columns [w D/8, (w+1) D/8). Phase 1 (projection y = res U)
+//    runs on tensor cores (mma.sync m16n8k16 bf16, fp32 accumulate) with U
+//    fragments read straight from global memory (L2-resident, shared by every
+//    CTA, fragment-ordered by the plan so each load is a coalesced 16-byte
+//    vector), two blocks ahead in registers. The eight partial y are summed in
+//    warp order in shared memory (deterministic);
+//  * phase 2 (re-projection): y split into bf16 hi + lo parts; V fragments
+//    stream like U; x arrives per warp through a ring of 64-column blocks
+//    (tensor copies), so the accumulators are finished as
+//    h = (res + x) + y V^T, rounded to bf16 and written over the residual;
+//  * the row amax is reduced across the 8 warps, then the h' tile leaves by
+//    2-D tensor stores while all threads pack the codes (coalesced 32-byte row
+//    segments per 8 lanes).
+// Each tensor copy or store is issued by its own lane: bulk copies from one
+// thread complete one after the other, copies from different threads overlap.
+// No wait is unbounded; a wait that gives up records a status code.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "boundary_kernels.cuh"
+#include "ptx.cuh"
+
+namespace respin {
+
+constexpr int kRtT = 16;                 // tokens per tile
+constexpr int kRtWarps = 8;
+constexpr int kRtThreads = kRtWarps * 32;
+constexpr int kRtBlockBytes = 2048;      // one 64-column block: 16 rows x 128 bytes
+
+template <int R>
+struct RtCfg {
+  static_assert(R == 16 || R == 32, "row-tile kernel: r <= 32");
+  static constexpr int XS = 4;             // x ring slots per warp
+  static constexpr int KK = R / 16;        // k16 steps of the re-projection
+  static constexpr int NT = R / 8;         // n8 tiles of y
+  static constexpr int UQ = R / 16;        // uint4 of U fragments per lane per k16 step
+  static constexpr int UB = 4 * UQ;        // ... per 64-column block (4 k16 steps)
+  static constexpr int VB = R / 4;         // uint4 of V fragments per lane per 64-column block
+  static constexpr int YP = R + 4;         // padded fp32 row of y
+  // shared-memory layout (offsets from a 1024-byte aligned base)
+  __host__ __device__ static constexpr uint32_t x_ring(int D) { return static_cast<uint32_t>(D) * 32; }
+  __host__ __device__ static constexpr uint32_t ypart(int D) { return x_ring(D) + kRtWarps * XS * kRtBlockBytes; }
+  __host__ __device__ static constexpr uint32_t ysum(int D) { return ypart(D) + kRtWarps * kRtT * YP * 4; }
+  __host__ __device__ static constexpr uint32_t wamax(int D) { return ysum(D) + kRtT * YP * 4; }
+  __host__ __device__ static constexpr uint32_t rowinv(int D) { return wamax(D) + kRtWarps * kRtT * 4; }
+  __host__ __device__ static constexpr uint32_t bars(int D) { return rowinv(D) + kRtT * 4; }
+  __host__ __device__ static constexpr uint32_t smem(int D) { return bars(D) + (kRtWarps + kRtWarps * XS) * 8 + 1024; }
+};
+
+// Byte offset of (row, 16-byte chunk c) inside a 64-column block in the
+// tensor-map 128-byte swizzle (chunk index XOR row mod 8).
+__device__ __forceinline__ uint32_t sw128(int row, int c) {
+  return static_cast<uint32_t>(row * 128 + ((c ^ (row & 7)) << 4));
+}
+
+__device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ void sts_u32(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint4 lds_u128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+
+// Component c (compile-time after unrolling) of a uint4.
+__device__ __forceinline__ uint32_t u4c(const uint4& v, int c) {
+  return c == 0 ? v.x : c == 1 ? v.y : c == 2 ? v.z : v.w;
+}
+
+// tmR / tmX / tmH: bf16 [N, D] tensor maps (residual, x, h'), box {64, 16},
+// 128-byte swizzle. Ut / Vt: U and V fragments in the order rt_pack_factors
+// writes. NB = D / 512 (64-column blocks per warp).
+template <int R, int NB, bool F32OUT>
+__global__ void __launch_bounds__(kRtThreads, 1)
+boundary_rowtile_kernel(const __grid_constant__ CUtensorMap tmR, const __grid_constant__ CUtensorMap tmX,
+                        const __grid_constant__ CUtensorMap tmH, const uint4* __restrict__ Ut,
+                        const uint4* __restrict__ Vt, int N, void* __restrict__ h_out,
+                        uint8_t* __restrict__ q_out, float* __restrict__ scale_out) {
+  using C = RtCfg<R>;
+  constexpr int XS = C::XS, D = NB * 512;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (base - raw);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, q4 = lane & 3;
+  const int ntiles = (N + kRtT - 1) / kRtT;
+  const uint32_t tileA = base;                       // block b at tileA + b * 2048
+  const uint32_t xring = base + C::x_ring(D);        // warp w, slot s at xring + (w XS + s) * 2048
+  float* ypart = reinterpret_cast<float*>(smem + C::ypart(D));
+  float* ysum = reinterpret_cast<float*>(smem + C::ysum(D));
+  float* wamax = reinterpret_cast<float*>(smem + C::wamax(D));
+  float* rowinv = reinterpret_cast<float*>(smem + C::rowinv(D));
+  const uint32_t res_bar = base + C::bars(D) + 8 * warp;                  // this warp's residual blocks
+  const uint32_t xbar0 = base + C::bars(D) + 8 * kRtWarps + 8 * warp * XS;  // this warp's x slots
+
+  if (tid == 0) {
+    for (int w = 0; w < kRtWarps; ++w) mbar_init(base + C::bars(D) + 8 * w, NB);
+    for (int i = 0; i < kRtWarps * XS; ++i) mbar_init(base + C::bars(D) + 8 * kRtWarps + 8 * i, 1);
+    fence_mbarrier_init();
+  }
+  __syncthreads();
+
+  // x block stream of this warp: use u is block u % NB of the warp's slice in
+  // its tile iteration u / NB, staged in slot u % XS by lane u % XS.
+  auto issue_x = [&](int u) {
+    const int tile = static_cast<int>(blockIdx.x) + (u / NB) * static_cast<int>(gridDim.x);
+    if (tile >= ntiles) return;
+    const int slot = u % XS;
+    mbar_arrive_expect_tx(xbar0 + 8 * slot, kRtBlockBytes);
+    tma_load_2d(xring + (warp * XS + slot) * kRtBlockBytes, &tmX, (warp * NB + u % NB) * 64, tile * kRtT,
+                xbar0 + 8 * slot);
+  };
+  if (lane < XS) issue_x(lane);
+
+  auto load_u = [&](uint4 (&dst)[C::UB], int j) {
+    const uint4* src = Ut + static_cast<size_t>(warp * NB + j) * C::UB * 32 + lane;
+#pragma unroll
+    for (int i = 0; i < C::UB; ++i) dst[i] = __ldg(src + i * 32);
+  };
+  auto load_v = [&](uint4 (&dst)[C::VB], int j) {
+    const uint4* src = Vt + static_cast<size_t>(warp * NB + j) * C::VB * 32 + lane;
+#pragma unroll
+    for (int i = 0; i < C::VB; ++i) dst[i] = __ldg(src + i * 32);
+  };
+
+  bool ok = true;
+  int it = 0;
+  for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
+    const int row0 = tile * kRtT;
+    // ---- residual tile: lane j < NB loads block warp * NB + j (after its
+    // own h' store of the previous tile has finished reading the block)
+    if (lane < NB) {
+      bulk_wait_group_read<0>();
+      const int b = warp * NB + lane;
+      mbar_arrive_expect_tx(res_bar, kRtBlockBytes);
+      tma_load_2d(tileA + b * kRtBlockBytes, &tmR, b * 64, row0, res_bar);
+    }
+
+    // ---- phase 1: partial y over this warp's columns
+    uint4 ub[3][C::UB];
+    load_u(ub[0], 0);
+    if (NB > 1) load_u(ub[1], 1);
+    float acc1[C::NT][4];
+#pragma unroll
+    for (int p = 0; p < C::NT; ++p) acc1[p][0] = acc1[p][1] = acc1[p][2] = acc1[p][3] = 0.f;
+    if (ok) ok = mbar_wait(res_bar, it & 1, kSiteBoundaryLoad);
+    ok = __all_sync(0xffffffffu, ok);
+#pragma unroll
+    for (int j = 0; j < NB; ++j) {
+      if (j + 2 < NB) load_u(ub[(j + 2) % 3], j + 2);
+      const uint32_t blk = tileA + (warp * NB + j) * kRtBlockBytes;
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const int row = (lane & 7) + 8 * ((lane >> 3) & 1);
+        uint32_t a[4];
+        ldmatrix_x4(blk + sw128(row, 2 * kk + (lane >> 4)), a[0], a[1], a[2], a[3]);
+#pragma unroll
+        for (int p = 0; p < C::NT; ++p) {
+          const uint4& v = ub[j % 3][kk * C::UQ + p / 2];
+          mma_bf16_16816(acc1[p], a, u4c(v, 2 * (p & 1)), u4c(v, 2 * (p & 1) + 1));
+        }
+      }
+    }
+    // V fragments of the first blocks load while y is reduced
+    uint4 vb[3][C::VB];
+    load_v(vb[0], 0);
+    if (NB > 1) load_v(vb[1], 1);
+    {
+      float* yp = ypart + warp * kRtT * C::YP;
+#pragma unroll
+      for (int p = 0; p < C::NT; ++p) {
+        *reinterpret_cast<float2*>(yp + g * C::YP + 8 * p + 2 * q4) = make_float2(acc1[p][0], acc1[p][1]);
+        *reinterpret_cast<float2*>(yp + (g + 8) * C::YP + 8 * p + 2 * q4) = make_float2(acc1[p][2], acc1[p][3]);
+      }
+    }
+    __syncthreads();
+    if (tid < kRtT * R / 2) {
+      const int row = tid / (R / 2), c2 = 2 * (tid % (R / 2));
+      float2 s = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int w = 0; w < kRtWarps; ++w) {
+        const float2 v = *reinterpret_cast<const float2*>(ypart + (w * kRtT + row) * C::YP + c2);
+        s.x += v.x;
+        s.y += v.y;
+      }
+      *reinterpret_cast<float2*>(ysum + row * C::YP + c2) = s;
+    }
+    __syncthreads();
+
+    // ---- phase 2: h = (res + x) + y V^T over this warp's columns
+    uint32_t ahi[C::KK][4], alo[C::KK][4];
+#pragma unroll
+    for (int kk = 0; kk < C::KK; ++kk) {
+      const float2 y0 = *reinterpret_cast<const float2*>(ysum + g * C::YP + 16 * kk + 2 * q4);
+      const float2 y1 = *reinterpret_cast<const float2*>(ysum + (g + 8) * C::YP + 16 * kk + 2 * q4);
+      const float2 y2 = *reinterpret_cast<const float2*>(ysum + g * C::YP + 16 * kk + 2 * q4 + 8);
+      const float2 y3 = *reinterpret_cast<const float2*>(ysum + (g + 8) * C::YP + 16 * kk + 2 * q4 + 8);
+      split_bf16x2(y0, ahi[kk][0], alo[kk][0]);
+      split_bf16x2(y1, ahi[kk][1], alo[kk][1]);
+      split_bf16x2(y2, ahi[kk][2], alo[kk][2]);
+      split_bf16x2(y3, ahi[kk][3], alo[kk][3]);
+    }
+    float rmax[2] = {0.f, 0.f};
+#pragma unroll
+    for (int j = 0; j < NB; ++j) {
+      if (j + 2 < NB) load_v(vb[(j + 2) % 3], j + 2);
+      const int u = it * NB + j;
+      const int slot = u % XS;
+      if (ok) ok = mbar_wait(xbar0 + 8 * slot, (u / XS) & 1, kSiteBoundaryLoad);
+      const uint32_t blk = tileA + (warp * NB + j) * kRtBlockBytes;
+      const uint32_t xblk = xring + (warp * XS + slot) * kRtBlockBytes;
+      const int colb = (warp * NB + j) * 64;
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int kk = 0; kk < C::KK; ++kk) {
+          const int ri = (t * C::KK + kk) * 2;
+          const uint4& v = vb[j % 3][ri / 4];
+          const uint32_t b0 = u4c(v, ri % 4), b1 = u4c(v, ri % 4 + 1);
+          mma_bf16_16816(acc, ahi[kk], b0, b1);
+          mma_bf16_16816(acc, alo[kk], b0, b1);
+        }
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const int row = g + 8 * hh;
+          const uint32_t off = sw128(row, t) + 4 * q4;
+          const uint32_t rw = lds_u32(blk + off), xw = lds_u32(xblk + off);
+          const float h0 = (bf16_lo_f32(rw) + bf16_lo_f32(xw)) + acc[2 * hh];
+          const float h1 = (bf16_hi_f32(rw) + bf16_hi_f32(xw)) + acc[2 * hh + 1];
+          const uint32_t hb = pack_bf16x2(h0, h1);
+          sts_u32(blk + off, hb);
+          rmax[hh] = fmaxf(rmax[hh], fmaxf(fabsf(bf16_lo_f32(hb)), fabsf(bf16_hi_f32(hb))));
+          if constexpr (F32OUT) {
+            if (h_out != nullptr && row0 + row < N)
+              *reinterpret_cast<float2*>(static_cast<float*>(h_out) + static_cast<size_t>(row0 + row) * D +
+                                         colb + 8 * t + 2 * q4) = make_float2(h0, h1);
+          }
+        }
+      }
+      // the slot's bytes were read (generic proxy) before its next tensor copy
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == slot) issue_x(u + XS);
+    }
+
+    // ---- row amax over the 8 warps, scales
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      float m = rmax[hh];
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+      if (q4 == 0) wamax[warp * kRtT + g + 8 * hh] = m;
+    }
+    fence_proxy_async_smem();   // h' in the tile (generic writes) before the tensor stores read it
+    __syncthreads();
+    if (tid < kRtT) {
+      float m = 0.f;
+#pragma unroll
+      for (int w = 0; w < kRtWarps; ++w) m = fmaxf(m, wamax[w * kRtT + tid]);
+      float inv, sc;
+      inv_and_scale(m, inv, sc);
+      rowinv[tid] = inv;
+      if (row0 + tid < N) scale_out[row0 + tid] = sc;
+    }
+    if constexpr (!F32OUT) {
+      if (h_out != nullptr && lane < NB) {
+        const int b = warp * NB + lane;
+        tma_store_2d(&tmH, b * 64, row0, tileA + b * kRtBlockBytes);
+        bulk_commit_group();
+      }
+    }
+    __syncthreads();
+
+    // ---- codes: chunk i = (block, row, 16-byte chunk); 8 lanes per row segment
+    constexpr int kChunks = kRtT * D / 8;
+#pragma unroll 4
+    for (int i = tid; i < kChunks; i += kRtThreads) {
+      const int b = i >> 7, row = (i >> 3) & 15, c = i & 7;
+      const uint4 hv = lds_u128(tileA + b * kRtBlockBytes + sw128(row, c));
+      const uint32_t code = quantize8_fast(hv, rowinv[row]);
+      if (ok && row0 + row < N)
+        reinterpret_cast<uint32_t*>(q_out)[static_cast<size_t>(row0 + row) * (D / 8) + b * 8 + c] = code;
+    }
+    fence_proxy_async_smem();   // these reads before the next residual copy into the tile
+    __syncthreads();
+  }
+  if (lane < NB) bulk_wait_group_all();
+}
+
+// Host side: U and V (bf16 bits, [D][R] row-major) in the fragment order of
+// boundary_rowtile_kernel. Ut: for 64-column block b, k16 step kk, lane
+// (g = lane / 4, q = lane % 4), register i = 2p + e of n8 tile p holds
+// (U[d][n], U[d+1][n]) with d = 64 b + 16 kk + 2q + 8e, n = 8p + g, stored at
+// uint4 ((b 4 + kk) R/16 + i/4) * 32 + lane, component i % 4. Vt: for block b,
+// register i = 2 (t R/16 + kk) + e holds (V[d][m], V[d][m+1]) with
+// d = 64 b + 8t + g, m = 16 kk + 2q + 8e, stored at uint4 (b R/4 + i/4) * 32 +
+// lane, component i % 4.
+inline void rt_pack_factors(const uint16_t* Ub, const uint16_t* Vb, int D, int R, uint32_t* Ut, uint32_t* Vt) {
+  auto pair = [](uint16_t lo, uint16_t hi) { return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16); };
+  const int UQ = R / 16, KK = R / 16, VB = R / 4;
+  for (int b = 0; b < D / 64; ++b)
+    for (int lane = 0; lane < 32; ++lane) {
+      const int g = lane >> 2, q = lane & 3;
+      for (int kk = 0; kk < 4; ++kk)
+        for (int i = 0; i < 4 * UQ; ++i) {
+          const int p = i / 2, e = i % 2;
+          const int d = 64 * b + 16 * kk + 2 * q + 8 * e, n = 8 * p + g;
+          const size_t idx = ((static_cast<size_t>(b * 4 + kk) * UQ + i / 4) * 32 + lane) * 4 + i % 4;
+          Ut[idx] = pair(Ub[static_cast<size_t>(d) * R + n], Ub[static_cast<size_t>(d + 1) * R + n]);
+        }
+      for (int i = 0; i < 4 * VB; ++i) {
+        const int e = i % 2, tk = i / 2, kk = tk % KK, t = tk / KK;
+        const int d = 64 * b + 8 * t + g, m = 16 * kk + 2 * q + 8 * e;
+        const size_t idx = ((static_cast<size_t>(b) * VB + i / 4) * 32 + lane) * 4 + i % 4;
+        Vt[idx] = pair(Vb[static_cast<size_t>(d) * R + m], Vb[static_cast<size_t>(d) * R + m + 1]);
+      }
+    }
+}
+
+}  // namespace respin

@@ -19,6 +19,7 @@
 #include "respin.h"
 #include "ptx.cuh"
 #include "boundary_kernels.cuh"
+#include "boundary_rowtile.cuh"
 #include "w4a4_gemm_kernels.cuh"
 
 using namespace respin;
@@ -60,7 +61,10 @@ bool aligned(const void* p, size_t a) {
 
 // ------------------------------------------------------------ plans
 
+enum BoundaryKind { kRowTile = 0, kClusterRf = 1, kClusterSmem = 2 };
+
 struct BoundaryConfig {
+  BoundaryKind kind = kClusterSmem;  // boundary_rowtile_kernel / cluster kernels
   bool rf = false;          // register-resident factors (boundary_cluster_rf_kernel)
   int T = 0, R = 0, cluster = 0, Dc = 0;
   size_t smem = 0;
@@ -86,6 +90,56 @@ std::set<respin_plan_s*> g_plans;
 bool plan_alive(respin_plan_s* p) {
   std::lock_guard<std::mutex> lk(g_plans_mu);
   return g_plans.count(p) != 0;
+}
+
+// cuTensorMapEncodeTiled, fetched once through the runtime's driver entry
+// point (no link-time dependency on the driver library).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_tiled() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+    cudaGetLastError();
+  });
+  return fn;
+}
+
+// 2-D bf16 tensor map over a row-major [rows, cols] matrix with a box of
+// 16 rows x 64 columns (128 bytes) in the 128-byte swizzle; rows past the end
+// read as zeros and are not written.
+bool make_tmap_bf16_tile(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols) {
+  EncodeTiledFn fn = encode_tiled();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * 2};
+  const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(kRtT)};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int R, int NB, bool F32>
+const void* rowtile_fn() {
+  return reinterpret_cast<const void*>(&boundary_rowtile_kernel<R, NB, F32>);
+}
+
+const void* pick_rowtile_fn(int R, int NB, bool f32) {
+#define RESPIN_PICK(RR, BB)                                                   \
+  if (R == RR && NB == BB) return f32 ? rowtile_fn<RR, BB, true>() : rowtile_fn<RR, BB, false>();
+  RESPIN_PICK(16, 2) RESPIN_PICK(16, 4) RESPIN_PICK(16, 8)
+  RESPIN_PICK(32, 2) RESPIN_PICK(32, 4) RESPIN_PICK(32, 8)
+#undef RESPIN_PICK
+  return nullptr;
 }
 
 template <int T, int R, bool F32>
@@ -168,6 +222,21 @@ respin_status_t configure_boundary(int D, int R, bool f32, BoundaryConfig* out) 
   int smem_optin = 0;
   e = cudaDeviceGetAttribute(&smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+  // Whole 16-token rows per CTA, factors streamed from L2 (no cluster).
+  if (R <= 32 && (D == 1024 || D == 2048 || D == 4096)) {
+    const size_t smem = R == 16 ? RtCfg<16>::smem(D) : RtCfg<32>::smem(D);
+    const void* fn = pick_rowtile_fn(R, D / 512, f32);
+    int sms = 0;
+    if (fn && smem <= static_cast<size_t>(smem_optin) &&
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess &&
+        cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) ==
+            cudaSuccess) {
+      out->kind = kRowTile; out->rf = false; out->T = kRtT; out->R = R; out->cluster = 1; out->Dc = D;
+      out->smem = smem; out->max_clusters = sms; out->fn = fn;
+      return ok();
+    }
+    cudaGetLastError();
+  }
   if (R <= 32) {
     for (int Dc : {1024, 512, 256}) {
       if (D % Dc || D / Dc > 16) continue;
@@ -177,7 +246,7 @@ respin_status_t configure_boundary(int D, int R, bool f32, BoundaryConfig* out) 
       const void* fn = pick_rf_fn(R, Dc, f32);
       const int n = max_active_clusters(fn, C, smem, kRfThreads);
       if (n <= 0) continue;
-      out->rf = true; out->T = kRfT; out->R = R; out->cluster = C; out->Dc = Dc;
+      out->kind = kClusterRf; out->rf = true; out->T = kRfT; out->R = R; out->cluster = C; out->Dc = Dc;
       out->smem = smem; out->max_clusters = n; out->fn = fn;
       return ok();
     }
@@ -194,7 +263,7 @@ respin_status_t configure_boundary(int D, int R, bool f32, BoundaryConfig* out) 
       if (smem > static_cast<size_t>(smem_optin)) continue;
       const int n = max_active_clusters(fn, C, smem, kBoundaryThreads);
       if (n <= 0) continue;
-      out->rf = false; out->T = T; out->R = R; out->cluster = C; out->Dc = Dc;
+      out->kind = kClusterSmem; out->rf = false; out->T = T; out->R = R; out->cluster = C; out->Dc = Dc;
       out->smem = smem; out->max_clusters = n; out->fn = fn;
       return ok();
     }
@@ -252,10 +321,13 @@ respin_status_t respin_plan_create(respin_plan_t* out, int D, int r, const float
         ub[static_cast<size_t>(d) * r_pad + j] = *reinterpret_cast<const uint16_t*>(&u);
         vb[static_cast<size_t>(d) * r_pad + j] = *reinterpret_cast<const uint16_t*>(&v);
       }
-    // Device layout: fragment order for the register-factor kernel, else
-    // U^T [r_pad, D] followed by V [D, r_pad].
+    // Device layout: fragment order for the row-tile and the register-factor
+    // kernels, else U^T [r_pad, D] followed by V [D, r_pad].
     std::vector<uint32_t> dev_words(static_cast<size_t>(D) * r_pad, 0);  // 2 * D * r_pad bf16
-    if (p->cfg.rf) {
+    if (p->cfg.kind == kRowTile) {
+      const size_t half = static_cast<size_t>(D) * r_pad / 2;
+      rt_pack_factors(ub.data(), vb.data(), D, r_pad, dev_words.data(), dev_words.data() + half);
+    } else if (p->cfg.rf) {
       const size_t half = static_cast<size_t>(D) * r_pad / 2;
       rf_pack_factors(ub.data(), vb.data(), D, r_pad, p->cfg.T, p->cfg.Dc, dev_words.data(), dev_words.data() + half);
     } else {
@@ -342,6 +414,20 @@ respin_status_t respin_boundary_forward(respin_plan_t plan, const void* x, const
 
   const BoundaryConfig& c = plan->cfg;
   const int ntiles = (N + c.T - 1) / c.T;
+  if (c.kind == kRowTile) {
+    CUtensorMap tmR, tmX, tmH;
+    const bool hmap = h_out != nullptr && !f32;
+    if (!make_tmap_bf16_tile(&tmR, residual, N, D) || !make_tmap_bf16_tile(&tmX, x, N, D) ||
+        !make_tmap_bf16_tile(&tmH, hmap ? h_out : residual, N, D))
+      return fail(RESPIN_ERR_CUDA, "cuTensorMapEncodeTiled failed for the boundary tiles");
+    const uint4* ut = reinterpret_cast<const uint4*>(plan->factors);
+    const uint4* vt = reinterpret_cast<const uint4*>(plan->factors + static_cast<size_t>(plan->r_pad) * D);
+    const int grid = ntiles < c.max_clusters ? ntiles : c.max_clusters;
+    void* args[] = {&tmR, &tmX, &tmH, &ut, &vt, &N, &h_out, &q_packed, &scale};
+    cudaError_t e = cudaLaunchKernel(c.fn, dim3(grid), dim3(kRtThreads), args, c.smem, s);
+    if (e != cudaSuccess) return cuda_fail(e, "boundary_rowtile_kernel launch");
+    return ok();
+  }
   const int nclusters = ntiles < c.max_clusters ? ntiles : c.max_clusters;
   cudaLaunchConfig_t lc = {};
   cudaLaunchAttribute attr[1];
@@ -421,27 +507,6 @@ static cudaError_t gemm_prepare(int dev, GemmDeviceInfo* info) {
   }
   *info = d;
   return cudaSuccess;
-}
-
-// cuTensorMapEncodeTiled, fetched once through the runtime's driver entry
-// point (no link-time dependency on the driver library).
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-static EncodeTiledFn encode_tiled() {
-  static EncodeTiledFn fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-    cudaGetLastError();
-  });
-  return fn;
 }
 
 // 2-D uint8 tensor map over a row-major [rows, cols] byte matrix with a box
