@@ -22,11 +22,13 @@
 //    stream like U; x arrives per warp through a ring of 64-column blocks
 //    (tensor copies), so the accumulators are finished as
 //    h = (res + x) + y V^T, rounded to bf16 and written over the residual;
-//  * the row amax is reduced across the 8 warps, then the h' tile leaves by
-//    2-D tensor stores while all threads pack the codes (coalesced 32-byte row
-//    segments per 8 lanes).
-// Each tensor copy or store is issued by its own lane: bulk copies from one
-// thread complete one after the other, copies from different threads overlap.
+//  * the row amax is reduced across the warps, then all threads read the h'
+//    tile once more in 16-byte chunks and write h' (128-byte row segments per
+//    8 lanes) and the packed codes (32-byte row segments per 8 lanes). A
+//    tensor store would hold its issuing thread for about 2 us on B200, longer
+//    than these plain stores take.
+// Each tensor copy is issued by its own lane: bulk copies from one thread
+// complete one after the other, copies from different threads overlap.
 // No wait is unbounded; a wait that gives up records a status code.
 #pragma once
 
@@ -40,14 +42,17 @@
 namespace respin {
 
 constexpr int kRtT = 16;                 // tokens per tile
-constexpr int kRtWarps = 8;
-constexpr int kRtThreads = kRtWarps * 32;
 constexpr int kRtBlockBytes = 2048;      // one 64-column block: 16 rows x 128 bytes
 
-template <int R>
+// W warps per CTA; warp w owns D / W columns (NB 64-column blocks).
+template <int R, int W>
 struct RtCfg {
   static_assert(R == 16 || R == 32, "row-tile kernel: r <= 32");
-  static constexpr int XS = 4;             // x ring slots per warp
+  static_assert(W == 8 || W == 16, "8 or 16 warps");
+  static constexpr int kWarps = W;
+  static constexpr int kThreads = 32 * W;
+  static constexpr int XS = W == 8 ? 4 : 2;      // x ring slots per warp
+  static constexpr int RING = W == 8 ? 3 : 2;    // factor fragments of RING blocks in registers
   static constexpr int KK = R / 16;        // k16 steps of the re-projection
   static constexpr int NT = R / 8;         // n8 tiles of y
   static constexpr int UQ = R / 16;        // uint4 of U fragments per lane per k16 step
@@ -56,12 +61,12 @@ struct RtCfg {
   static constexpr int YP = R + 4;         // padded fp32 row of y
   // shared-memory layout (offsets from a 1024-byte aligned base)
   __host__ __device__ static constexpr uint32_t x_ring(int D) { return static_cast<uint32_t>(D) * 32; }
-  __host__ __device__ static constexpr uint32_t ypart(int D) { return x_ring(D) + kRtWarps * XS * kRtBlockBytes; }
-  __host__ __device__ static constexpr uint32_t ysum(int D) { return ypart(D) + kRtWarps * kRtT * YP * 4; }
+  __host__ __device__ static constexpr uint32_t ypart(int D) { return x_ring(D) + W * XS * kRtBlockBytes; }
+  __host__ __device__ static constexpr uint32_t ysum(int D) { return ypart(D) + W * kRtT * YP * 4; }
   __host__ __device__ static constexpr uint32_t wamax(int D) { return ysum(D) + kRtT * YP * 4; }
-  __host__ __device__ static constexpr uint32_t rowinv(int D) { return wamax(D) + kRtWarps * kRtT * 4; }
+  __host__ __device__ static constexpr uint32_t rowinv(int D) { return wamax(D) + W * kRtT * 4; }
   __host__ __device__ static constexpr uint32_t bars(int D) { return rowinv(D) + kRtT * 4; }
-  __host__ __device__ static constexpr uint32_t smem(int D) { return bars(D) + (kRtWarps + kRtWarps * XS) * 8 + 1024; }
+  __host__ __device__ static constexpr uint32_t smem(int D) { return bars(D) + (W + W * XS) * 8 + 1024; }
 };
 
 // Byte offset of (row, 16-byte chunk c) inside a 64-column block in the
@@ -70,36 +75,75 @@ __device__ __forceinline__ uint32_t sw128(int row, int c) {
   return static_cast<uint32_t>(row * 128 + ((c ^ (row & 7)) << 4));
 }
 
-__device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
-  uint32_t v;
-  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
-  return v;
-}
-__device__ __forceinline__ void sts_u32(uint32_t addr, uint32_t v) {
-  asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
-}
-__device__ __forceinline__ uint4 lds_u128(uint32_t addr) {
-  uint4 v;
-  asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
-  return v;
-}
-
 // Component c (compile-time after unrolling) of a uint4.
 __device__ __forceinline__ uint32_t u4c(const uint4& v, int c) {
   return c == 0 ? v.x : c == 1 ? v.y : c == 2 ? v.z : v.w;
 }
 
-// tmR / tmX / tmH: bf16 [N, D] tensor maps (residual, x, h'), box {64, 16},
-// 128-byte swizzle. Ut / Vt: U and V fragments in the order rt_pack_factors
+// Paired binary32 arithmetic (sm_100 f32x2): each lane rounds exactly as the
+// scalar operation would, so results equal the scalar sequence.
+__device__ __forceinline__ float2 add_f32x2(float2 a, float2 b) {
+  float2 r;
+  asm("{\n\t.reg .b64 a, b, r;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+      "add.rn.f32x2 r, a, b;\n\tmov.b64 {%0, %1}, r;\n\t}"
+      : "=f"(r.x), "=f"(r.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return r;
+}
+__device__ __forceinline__ float2 mul_f32x2(float2 a, float2 b) {
+  float2 r;
+  asm("{\n\t.reg .b64 a, b, r;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+      "mul.rn.f32x2 r, a, b;\n\tmov.b64 {%0, %1}, r;\n\t}"
+      : "=f"(r.x), "=f"(r.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return r;
+}
+// Running maximum of |v| over both bf16 halves (bf16 values are compared
+// exactly; a NaN operand is ignored like fmaxf does).
+__device__ __forceinline__ uint32_t absmax_bf16x2(uint32_t m, uint32_t v) {
+  uint32_t r;
+  asm("{\n\t.reg .b32 t;\n\tabs.bf16x2 t, %2;\n\tmax.bf16x2 %0, %1, t;\n\t}" : "=r"(r) : "r"(m), "r"(v));
+  return r;
+}
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+  return r;
+}
+__device__ __forceinline__ float2 bf16x2_to_f32x2(uint32_t w) {
+  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+
+// 8 bf16 values -> 8 packed INT4 codes (as quantize8_fast): u = fl(fl(g inv)
+// + 1.5 2^23) keeps rint(g inv) in its low byte (two's complement, since
+// |g inv| < 8); the low bytes are gathered with byte permutes and their low
+// nibbles packed, element e at bits 4e..4e+3. The products are paired; the
+// additions are scalar __fadd_rn, because a paired add after a paired
+// multiply may be contracted into a fused multiply-add, which skips the
+// binary32 rounding of g inv (measured: 7 codes in 2^20 differ).
+__device__ __forceinline__ uint32_t quantize8_x2(const uint4 hv, float inv) {
+  const float2 iv = make_float2(inv, inv);
+  const float2 p0 = mul_f32x2(bf16x2_to_f32x2(hv.x), iv), p1 = mul_f32x2(bf16x2_to_f32x2(hv.y), iv);
+  const float2 p2 = mul_f32x2(bf16x2_to_f32x2(hv.z), iv), p3 = mul_f32x2(bf16x2_to_f32x2(hv.w), iv);
+  auto u = [](float v) { return __float_as_uint(__fadd_rn(v, 12582912.0f)); };
+  // bytes [c0 c1 c2 c3] and [c4 c5 c6 c7]
+  const uint32_t w0 = prmt(prmt(u(p0.x), u(p0.y), 0x0040u), prmt(u(p1.x), u(p1.y), 0x0040u), 0x5410u);
+  const uint32_t w1 = prmt(prmt(u(p2.x), u(p2.y), 0x0040u), prmt(u(p3.x), u(p3.y), 0x0040u), 0x5410u);
+  // byte 0 <- c0 | c1 << 4, byte 2 <- c2 | c3 << 4 (bytes 1, 3 unused)
+  const uint32_t y0 = (w0 & 0x000F000Fu) | ((w0 >> 4) & 0x00F000F0u);
+  const uint32_t y1 = (w1 & 0x000F000Fu) | ((w1 >> 4) & 0x00F000F0u);
+  return prmt(y0, y1, 0x6420u);
+}
+
+// tmR / tmX: bf16 [N, D] tensor maps (residual, x), box {64, 16}, 128-byte
+// swizzle. Ut / Vt: U and V fragments in the order rt_pack_factors
 // writes. NB = D / 512 (64-column blocks per warp).
-template <int R, int NB, bool F32OUT>
-__global__ void __launch_bounds__(kRtThreads, 1)
+template <int R, int W, int NB, bool F32OUT>
+__global__ void __launch_bounds__(32 * W, 1)
 boundary_rowtile_kernel(const __grid_constant__ CUtensorMap tmR, const __grid_constant__ CUtensorMap tmX,
-                        const __grid_constant__ CUtensorMap tmH, const uint4* __restrict__ Ut,
+                        const uint4* __restrict__ Ut,
                         const uint4* __restrict__ Vt, int N, void* __restrict__ h_out,
                         uint8_t* __restrict__ q_out, float* __restrict__ scale_out) {
-  using C = RtCfg<R>;
-  constexpr int XS = C::XS, D = NB * 512;
+  using C = RtCfg<R, W>;
+  constexpr int XS = C::XS, RING = C::RING, D = NB * 64 * W;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -114,14 +158,20 @@ boundary_rowtile_kernel(const __grid_constant__ CUtensorMap tmR, const __grid_co
   float* wamax = reinterpret_cast<float*>(smem + C::wamax(D));
   float* rowinv = reinterpret_cast<float*>(smem + C::rowinv(D));
   const uint32_t res_bar = base + C::bars(D) + 8 * warp;                  // this warp's residual blocks
-  const uint32_t xbar0 = base + C::bars(D) + 8 * kRtWarps + 8 * warp * XS;  // this warp's x slots
+  const uint32_t xbar0 = base + C::bars(D) + 8 * W + 8 * warp * XS;  // this warp's x slots
 
-  if (tid == 0) {
-    for (int w = 0; w < kRtWarps; ++w) mbar_init(base + C::bars(D) + 8 * w, NB);
-    for (int i = 0; i < kRtWarps * XS; ++i) mbar_init(base + C::bars(D) + 8 * kRtWarps + 8 * i, 1);
+  // Each warp initialises its own barriers and starts its copies at once (no
+  // CTA-wide barrier before the first tensor copy).
+  if (lane == 0) {
+    mbar_init(res_bar, NB);
+    for (int i = 0; i < XS; ++i) mbar_init(xbar0 + 8 * i, 1);
     fence_mbarrier_init();
+    if (warp == 0) {
+      asm volatile("prefetch.tensormap [%0];" ::"l"(&tmR) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"(&tmX) : "memory");
+    }
   }
-  __syncthreads();
+  __syncwarp();
 
   // x block stream of this warp: use u is block u % NB of the warp's slice in
   // its tile iteration u / NB, staged in slot u % XS by lane u % XS.
@@ -153,16 +203,16 @@ boundary_rowtile_kernel(const __grid_constant__ CUtensorMap tmR, const __grid_co
     // ---- residual tile: lane j < NB loads block warp * NB + j (after its
     // own h' store of the previous tile has finished reading the block)
     if (lane < NB) {
-      bulk_wait_group_read<0>();
       const int b = warp * NB + lane;
       mbar_arrive_expect_tx(res_bar, kRtBlockBytes);
       tma_load_2d(tileA + b * kRtBlockBytes, &tmR, b * 64, row0, res_bar);
     }
 
     // ---- phase 1: partial y over this warp's columns
-    uint4 ub[3][C::UB];
-    load_u(ub[0], 0);
-    if (NB > 1) load_u(ub[1], 1);
+    uint4 ub[RING][C::UB];
+#pragma unroll
+    for (int j = 0; j < RING - 1; ++j)
+      if (j < NB) load_u(ub[j], j);
     float acc1[C::NT][4];
 #pragma unroll
     for (int p = 0; p < C::NT; ++p) acc1[p][0] = acc1[p][1] = acc1[p][2] = acc1[p][3] = 0.f;
@@ -170,7 +220,7 @@ boundary_rowtile_kernel(const __grid_constant__ CUtensorMap tmR, const __grid_co
     ok = __all_sync(0xffffffffu, ok);
 #pragma unroll
     for (int j = 0; j < NB; ++j) {
-      if (j + 2 < NB) load_u(ub[(j + 2) % 3], j + 2);
+      if (j + RING - 1 < NB) load_u(ub[(j + RING - 1) % RING], j + RING - 1);
       const uint32_t blk = tileA + (warp * NB + j) * kRtBlockBytes;
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk) {
@@ -179,15 +229,16 @@ boundary_rowtile_kernel(const __grid_constant__ CUtensorMap tmR, const __grid_co
         ldmatrix_x4(blk + sw128(row, 2 * kk + (lane >> 4)), a[0], a[1], a[2], a[3]);
 #pragma unroll
         for (int p = 0; p < C::NT; ++p) {
-          const uint4& v = ub[j % 3][kk * C::UQ + p / 2];
+          const uint4& v = ub[j % RING][kk * C::UQ + p / 2];
           mma_bf16_16816(acc1[p], a, u4c(v, 2 * (p & 1)), u4c(v, 2 * (p & 1) + 1));
         }
       }
     }
     // V fragments of the first blocks load while y is reduced
-    uint4 vb[3][C::VB];
-    load_v(vb[0], 0);
-    if (NB > 1) load_v(vb[1], 1);
+    uint4 vb[RING][C::VB];
+#pragma unroll
+    for (int j = 0; j < RING - 1; ++j)
+      if (j < NB) load_v(vb[j], j);
     {
       float* yp = ypart + warp * kRtT * C::YP;
 #pragma unroll
@@ -201,7 +252,7 @@ boundary_rowtile_kernel(const __grid_constant__ CUtensorMap tmR, const __grid_co
       const int row = tid / (R / 2), c2 = 2 * (tid % (R / 2));
       float2 s = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int w = 0; w < kRtWarps; ++w) {
+      for (int w = 0; w < W; ++w) {
         const float2 v = *reinterpret_cast<const float2*>(ypart + (w * kRtT + row) * C::YP + c2);
         s.x += v.x;
         s.y += v.y;
@@ -223,41 +274,57 @@ boundary_rowtile_kernel(const __grid_constant__ CUtensorMap tmR, const __grid_co
       split_bf16x2(y2, ahi[kk][2], alo[kk][2]);
       split_bf16x2(y3, ahi[kk][3], alo[kk][3]);
     }
-    float rmax[2] = {0.f, 0.f};
+    uint32_t amax2[2] = {0u, 0u};   // running max |h'| (bf16x2) of rows g and g + 8
+    // (row, chunk t) -> row * 128 + ((t ^ row % 8) << 4): the XOR only touches
+    // bits 4-6, which are zero in row * 128 + 4 q4, so it folds into one XOR.
+    const uint32_t rb[2] = {static_cast<uint32_t>(g * 128 + 4 * q4 + (g << 4)),
+                            static_cast<uint32_t>((g + 8) * 128 + 4 * q4 + (g << 4))};
 #pragma unroll
     for (int j = 0; j < NB; ++j) {
-      if (j + 2 < NB) load_v(vb[(j + 2) % 3], j + 2);
+      if (j + RING - 1 < NB) load_v(vb[(j + RING - 1) % RING], j + RING - 1);
       const int u = it * NB + j;
       const int slot = u % XS;
       if (ok) ok = mbar_wait(xbar0 + 8 * slot, (u / XS) & 1, kSiteBoundaryLoad);
-      const uint32_t blk = tileA + (warp * NB + j) * kRtBlockBytes;
-      const uint32_t xblk = xring + (warp * XS + slot) * kRtBlockBytes;
+      uint8_t* blk = smem + (warp * NB + j) * kRtBlockBytes;
+      const uint8_t* xblk = smem + C::x_ring(D) + (warp * XS + slot) * kRtBlockBytes;
       const int colb = (warp * NB + j) * 64;
+      // all MMAs of the block first (8 independent accumulators), then the
+      // epilogue; per accumulator the order is hi, lo per k16 step
+      float acc[8][4];
 #pragma unroll
-      for (int t = 0; t < 8; ++t) {
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int t = 0; t < 8; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
 #pragma unroll
-        for (int kk = 0; kk < C::KK; ++kk) {
+      for (int kk = 0; kk < C::KK; ++kk) {
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
           const int ri = (t * C::KK + kk) * 2;
-          const uint4& v = vb[j % 3][ri / 4];
-          const uint32_t b0 = u4c(v, ri % 4), b1 = u4c(v, ri % 4 + 1);
-          mma_bf16_16816(acc, ahi[kk], b0, b1);
-          mma_bf16_16816(acc, alo[kk], b0, b1);
+          const uint4& v = vb[j % RING][ri / 4];
+          mma_bf16_16816(acc[t], ahi[kk], u4c(v, ri % 4), u4c(v, ri % 4 + 1));
         }
 #pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          const int ri = (t * C::KK + kk) * 2;
+          const uint4& v = vb[j % RING][ri / 4];
+          mma_bf16_16816(acc[t], alo[kk], u4c(v, ri % 4), u4c(v, ri % 4 + 1));
+        }
+      }
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+#pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
-          const int row = g + 8 * hh;
-          const uint32_t off = sw128(row, t) + 4 * q4;
-          const uint32_t rw = lds_u32(blk + off), xw = lds_u32(xblk + off);
-          const float h0 = (bf16_lo_f32(rw) + bf16_lo_f32(xw)) + acc[2 * hh];
-          const float h1 = (bf16_hi_f32(rw) + bf16_hi_f32(xw)) + acc[2 * hh + 1];
-          const uint32_t hb = pack_bf16x2(h0, h1);
-          sts_u32(blk + off, hb);
-          rmax[hh] = fmaxf(rmax[hh], fmaxf(fabsf(bf16_lo_f32(hb)), fabsf(bf16_hi_f32(hb))));
+          const uint32_t off = rb[hh] ^ static_cast<uint32_t>(t << 4);
+          const uint32_t rw = *reinterpret_cast<const uint32_t*>(blk + off);
+          const uint32_t xw = *reinterpret_cast<const uint32_t*>(xblk + off);
+          const float2 sum = add_f32x2(bf16x2_to_f32x2(rw), bf16x2_to_f32x2(xw));
+          const float2 h = add_f32x2(sum, make_float2(acc[t][2 * hh], acc[t][2 * hh + 1]));
+          const uint32_t hb = pack_bf16x2(h.x, h.y);
+          *reinterpret_cast<uint32_t*>(blk + off) = hb;
+          amax2[hh] = absmax_bf16x2(amax2[hh], hb);
           if constexpr (F32OUT) {
+            const int row = g + 8 * hh;
             if (h_out != nullptr && row0 + row < N)
               *reinterpret_cast<float2*>(static_cast<float*>(h_out) + static_cast<size_t>(row0 + row) * D +
-                                         colb + 8 * t + 2 * q4) = make_float2(h0, h1);
+                                         colb + 8 * t + 2 * q4) = h;
           }
         }
       }
@@ -266,6 +333,9 @@ boundary_rowtile_kernel(const __grid_constant__ CUtensorMap tmR, const __grid_co
       __syncwarp();
       if (lane == slot) issue_x(u + XS);
     }
+    float rmax[2];
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) rmax[hh] = fmaxf(bf16_lo_f32(amax2[hh]), bf16_hi_f32(amax2[hh]));
 
     // ---- row amax over the 8 warps, scales
 #pragma unroll
@@ -275,40 +345,38 @@ boundary_rowtile_kernel(const __grid_constant__ CUtensorMap tmR, const __grid_co
       m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
       if (q4 == 0) wamax[warp * kRtT + g + 8 * hh] = m;
     }
-    fence_proxy_async_smem();   // h' in the tile (generic writes) before the tensor stores read it
     __syncthreads();
     if (tid < kRtT) {
       float m = 0.f;
 #pragma unroll
-      for (int w = 0; w < kRtWarps; ++w) m = fmaxf(m, wamax[w * kRtT + tid]);
+      for (int w = 0; w < W; ++w) m = fmaxf(m, wamax[w * kRtT + tid]);
       float inv, sc;
       inv_and_scale(m, inv, sc);
       rowinv[tid] = inv;
       if (row0 + tid < N) scale_out[row0 + tid] = sc;
     }
-    if constexpr (!F32OUT) {
-      if (h_out != nullptr && lane < NB) {
-        const int b = warp * NB + lane;
-        tma_store_2d(&tmH, b * 64, row0, tileA + b * kRtBlockBytes);
-        bulk_commit_group();
-      }
-    }
     __syncthreads();
 
-    // ---- codes: chunk i = (block, row, 16-byte chunk); 8 lanes per row segment
+    // ---- h' out and codes: chunk i = (block, row, 16-byte chunk); 8 lanes
+    // write one 128-byte h' row segment and one 32-byte code segment
     constexpr int kChunks = kRtT * D / 8;
 #pragma unroll 4
-    for (int i = tid; i < kChunks; i += kRtThreads) {
+    for (int i = tid; i < kChunks; i += C::kThreads) {
       const int b = i >> 7, row = (i >> 3) & 15, c = i & 7;
-      const uint4 hv = lds_u128(tileA + b * kRtBlockBytes + sw128(row, c));
-      const uint32_t code = quantize8_fast(hv, rowinv[row]);
-      if (ok && row0 + row < N)
-        reinterpret_cast<uint32_t*>(q_out)[static_cast<size_t>(row0 + row) * (D / 8) + b * 8 + c] = code;
+      const uint4 hv = *reinterpret_cast<const uint4*>(smem + b * kRtBlockBytes + sw128(row, c));
+      const uint32_t code = quantize8_x2(hv, rowinv[row]);
+      if (ok && row0 + row < N) {
+        const size_t grow = static_cast<size_t>(row0 + row);
+        reinterpret_cast<uint32_t*>(q_out)[grow * (D / 8) + b * 8 + c] = code;
+        if constexpr (!F32OUT) {
+          if (h_out != nullptr)
+            *reinterpret_cast<uint4*>(static_cast<bf16*>(h_out) + grow * D + b * 64 + c * 8) = hv;
+        }
+      }
     }
     fence_proxy_async_smem();   // these reads before the next residual copy into the tile
     __syncthreads();
   }
-  if (lane < NB) bulk_wait_group_all();
 }
 
 // Host side: U and V (bf16 bits, [D][R] row-major) in the fragment order of

@@ -281,10 +281,12 @@ __device__ __forceinline__ void ldmatrix_x2(uint32_t addr, uint32_t& r0, uint32_
                : "r"(addr));
 }
 
-// D += A * B, m16n8k16, bf16 inputs, fp32 accumulate.
+// D += A * B, m16n8k16, bf16 inputs, fp32 accumulate. A pure function of its
+// register operands (not volatile), so the compiler may interleave
+// independent MMAs with loads and other work.
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4],
                                                uint32_t b0, uint32_t b1) {
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
       "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])

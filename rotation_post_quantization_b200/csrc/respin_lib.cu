@@ -115,7 +115,7 @@ static EncodeTiledFn encode_tiled() {
 
 // 2-D bf16 tensor map over a row-major [rows, cols] matrix with a box of
 // 16 rows x 64 columns (128 bytes) in the 128-byte swizzle; rows past the end
-// read as zeros and are not written.
+// read as zeros.
 bool make_tmap_bf16_tile(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols) {
   EncodeTiledFn fn = encode_tiled();
   if (!fn) return false;
@@ -128,18 +128,32 @@ bool make_tmap_bf16_tile(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int R, int NB, bool F32>
+template <int R, int W, int NB, bool F32>
 const void* rowtile_fn() {
-  return reinterpret_cast<const void*>(&boundary_rowtile_kernel<R, NB, F32>);
+  return reinterpret_cast<const void*>(&boundary_rowtile_kernel<R, W, NB, F32>);
 }
 
-const void* pick_rowtile_fn(int R, int NB, bool f32) {
-#define RESPIN_PICK(RR, BB)                                                   \
-  if (R == RR && NB == BB) return f32 ? rowtile_fn<RR, BB, true>() : rowtile_fn<RR, BB, false>();
-  RESPIN_PICK(16, 2) RESPIN_PICK(16, 4) RESPIN_PICK(16, 8)
-  RESPIN_PICK(32, 2) RESPIN_PICK(32, 4) RESPIN_PICK(32, 8)
+// Warps per CTA of the row-tile kernel for a given D (16 where D / 16 still
+// holds whole 64-column blocks, for more latency hiding per SM).
+#ifndef RESPIN_RT_WARPS
+#define RESPIN_RT_WARPS 8
+#endif
+int rowtile_warps(int D) { return RESPIN_RT_WARPS == 16 && D >= 2048 ? 16 : 8; }
+
+const void* pick_rowtile_fn(int R, int D, bool f32) {
+  const int W = rowtile_warps(D), NB = D / (64 * W);
+#define RESPIN_PICK(RR, WW, BB) \
+  if (R == RR && W == WW && NB == BB) return f32 ? rowtile_fn<RR, WW, BB, true>() : rowtile_fn<RR, WW, BB, false>();
+  RESPIN_PICK(16, 8, 2) RESPIN_PICK(16, 8, 4) RESPIN_PICK(16, 8, 8) RESPIN_PICK(16, 16, 2) RESPIN_PICK(16, 16, 4)
+  RESPIN_PICK(32, 8, 2) RESPIN_PICK(32, 8, 4) RESPIN_PICK(32, 8, 8) RESPIN_PICK(32, 16, 2) RESPIN_PICK(32, 16, 4)
 #undef RESPIN_PICK
   return nullptr;
+}
+
+size_t rowtile_smem(int R, int D) {
+  const int W = rowtile_warps(D);
+  if (R == 16) return W == 16 ? RtCfg<16, 16>::smem(D) : RtCfg<16, 8>::smem(D);
+  return W == 16 ? RtCfg<32, 16>::smem(D) : RtCfg<32, 8>::smem(D);
 }
 
 template <int T, int R, bool F32>
@@ -224,14 +238,14 @@ respin_status_t configure_boundary(int D, int R, bool f32, BoundaryConfig* out) 
   if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
   // Whole 16-token rows per CTA, factors streamed from L2 (no cluster).
   if (R <= 32 && (D == 1024 || D == 2048 || D == 4096)) {
-    const size_t smem = R == 16 ? RtCfg<16>::smem(D) : RtCfg<32>::smem(D);
-    const void* fn = pick_rowtile_fn(R, D / 512, f32);
+    const size_t smem = rowtile_smem(R, D);
+    const void* fn = pick_rowtile_fn(R, D, f32);
     int sms = 0;
     if (fn && smem <= static_cast<size_t>(smem_optin) &&
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess &&
         cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) ==
             cudaSuccess) {
-      out->kind = kRowTile; out->rf = false; out->T = kRtT; out->R = R; out->cluster = 1; out->Dc = D;
+      out->kind = kRowTile; out->rf = false; out->T = kRtT; out->R = R; out->cluster = rowtile_warps(D); out->Dc = D;
       out->smem = smem; out->max_clusters = sms; out->fn = fn;
       return ok();
     }
@@ -415,16 +429,14 @@ respin_status_t respin_boundary_forward(respin_plan_t plan, const void* x, const
   const BoundaryConfig& c = plan->cfg;
   const int ntiles = (N + c.T - 1) / c.T;
   if (c.kind == kRowTile) {
-    CUtensorMap tmR, tmX, tmH;
-    const bool hmap = h_out != nullptr && !f32;
-    if (!make_tmap_bf16_tile(&tmR, residual, N, D) || !make_tmap_bf16_tile(&tmX, x, N, D) ||
-        !make_tmap_bf16_tile(&tmH, hmap ? h_out : residual, N, D))
+    CUtensorMap tmR, tmX;
+    if (!make_tmap_bf16_tile(&tmR, residual, N, D) || !make_tmap_bf16_tile(&tmX, x, N, D))
       return fail(RESPIN_ERR_CUDA, "cuTensorMapEncodeTiled failed for the boundary tiles");
     const uint4* ut = reinterpret_cast<const uint4*>(plan->factors);
     const uint4* vt = reinterpret_cast<const uint4*>(plan->factors + static_cast<size_t>(plan->r_pad) * D);
     const int grid = ntiles < c.max_clusters ? ntiles : c.max_clusters;
-    void* args[] = {&tmR, &tmX, &tmH, &ut, &vt, &N, &h_out, &q_packed, &scale};
-    cudaError_t e = cudaLaunchKernel(c.fn, dim3(grid), dim3(kRtThreads), args, c.smem, s);
+    void* args[] = {&tmR, &tmX, &ut, &vt, &N, &h_out, &q_packed, &scale};
+    cudaError_t e = cudaLaunchKernel(c.fn, dim3(grid), dim3(32 * c.cluster), args, c.smem, s);
     if (e != cudaSuccess) return cuda_fail(e, "boundary_rowtile_kernel launch");
     return ok();
   }
