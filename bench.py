@@ -234,6 +234,49 @@ def traffic_for(kernel_file: str, name: str):
     return None
 
 
+# ---------------------------------------------------------------- ranks
+
+def rank_env():
+    """(rank, world size, local rank) from the torchrun environment."""
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def init_dist(backend: str, device=None, timeout_s: float = 120.0):
+    """Process group for the barrier and the max-over-ranks reduction; a short
+    timeout so that ranks waiting for a dead peer end with an error."""
+    import datetime
+    import torch.distributed as dist
+    kw = dict(timeout=datetime.timedelta(seconds=timeout_s))
+    if device is not None:
+        kw["device_id"] = device
+    dist.init_process_group(backend, **kw)
+    return dist
+
+
+def max_over_ranks(values, dist, device=None):
+    """Element-wise maximum of per-rank timings (every rank gets the result);
+    the identity without a process group."""
+    import torch
+    if dist is None:
+        return list(values)
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_tokens_per_s(world: int, tokens_per_rank: int, ms_per_step: float) -> float:
+    """Whole-job throughput under weak scaling: every rank processes its own
+    tokens_per_rank tokens per step, the step lasts the slowest rank's time."""
+    return world * tokens_per_rank / (ms_per_step * 1e-3)
+
+
+def rank_seed(rank: int, i: int) -> int:
+    """Seed of input set i on a rank: ranks hold different tokens (shards of
+    the batch), set i of rank 0 is the workload's own fixture."""
+    return 1000 * rank + i
+
+
 # ---------------------------------------------------------------- our arm
 
 def run_ours(args, rank: int, world: int, local_rank: int):
@@ -244,12 +287,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    dist = None
-    if world > 1:
-        import torch.distributed as dist
-        import datetime
-        dist.init_process_group("nccl", device_id=dev,
-                                timeout=datetime.timedelta(seconds=120))
+    dist = init_dist("nccl", dev) if world > 1 else None
 
     w, fx, qw_np, sw_np = workload_inputs("cuda")
     D, N, r, O_ = w.D, w.N, w.r, w.O
@@ -259,7 +297,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     sets = []
     for i in range(NSETS):
         kw = dict(n_outlier=w.n_outlier, outlier_scale=w.outlier_scale,
-                  dist=w.dist, seed=1000 * rank + i)
+                  dist=w.dist, seed=rank_seed(rank, i))
         x = W.activations_bf16_fast(N, D, tensor_id=W.TID_X, device=str(dev), **kw)
         res = W.activations_bf16_fast(N, D, tensor_id=W.TID_RESIDUAL,
                                       device=str(dev), **kw)
@@ -356,11 +394,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     e2e_ms = e0.elapsed_time(e1) / Ke
     sampler.stop_evt.set()
 
-    times = torch.tensor([total_ms, e2e_ms, b_ms, g_ms], dtype=torch.float64,
-                         device=dev)
-    if dist:
-        dist.all_reduce(times, op=dist.ReduceOp.MAX)
-    total_ms, e2e_ms, b_ms, g_ms = times.tolist()
+    total_ms, e2e_ms, b_ms, g_ms = max_over_ranks([total_ms, e2e_ms, b_ms, g_ms],
+                                                  dist, dev)
     ms_step = total_ms / Ksteps
 
     if rank == 0:
@@ -372,14 +407,14 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         b_gbs = b_bytes / (b_ms * 1e-3) / 1e9
         line = {
             "metric": METRIC,
-            "value": world * N / (ms_step * 1e-3),
+            "value": job_tokens_per_s(world, N, ms_step),
             "unit": "tokens/s",
             "n_gpus": world, "steps": Ksteps, "warmup": args.warmup,
             "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16+int4", "data": "synthetic",
             "config": config_block(w, world),
-            "boundary_tokens_per_s": world * N / (b_ms * 1e-3),
+            "boundary_tokens_per_s": job_tokens_per_s(world, N, b_ms),
             "boundary_us": b_ms * 1e3,
             "gemm_tops": gemm_tops * world,
             "gemm_us": g_ms * 1e3,
@@ -399,7 +434,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                 "traffic": traffic_for("boundary_rowtile.cuh",
                                        "boundary_rowtile_kernel"),
                 "peak_source": "%s HBM copy bandwidth" % src},
-            "e2e": {"value": world * N / (e2e_ms * 1e-3), "unit": "tokens/s",
+            "e2e": {"value": job_tokens_per_s(world, N, e2e_ms), "unit": "tokens/s",
                     "h2d_bytes_per_step": 2 * N * D * 2,
                     "d2h_bytes_per_step": N * O_ * 2 + N * D * 2},
             "gpu_launches": 2 * Ksteps,
@@ -453,9 +488,7 @@ def main():
     if args.profile_launch:
         run_profile_launch(args)
         return
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    rank, world, local_rank = rank_env()
     if args.impl == "reference":
         run_reference(args, rank)
         return
