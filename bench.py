@@ -48,6 +48,11 @@ def parse_args():
                         "(for ncu captures); prints no bench line")
     p.add_argument("--tokens", type=int, default=None,
                    help="tokens for --profile-launch (default 2048)")
+    p.add_argument("--workload", default="llama2_7b",
+                   choices=["llama2_7b", "tiny", "decode", "llama2_70b", "llama3_8b_stack"],
+                   help="llama2_7b (default): the headline step. The others print "
+                        "one JSON line each for the remaining workload configurations "
+                        "(1 GPU)")
     return p.parse_args()
 
 
@@ -449,6 +454,209 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         dist.destroy_process_group()
 
 
+# ---------------------------------------------------------------- other workloads
+
+def _events_ms(torch, fn, iters: int, stream) -> float:
+    """Mean device time of fn() over iters launches (CUDA events on `stream`)."""
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for i in range(iters):
+        fn(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / iters
+
+
+def _plan_for(rq, W, D, r, k, nu, seed=0):
+    import numpy as np
+    Q = W.orthonormal_basis(D, k, seed)
+    U, V = W.lowrank_factors(Q, W.plane_angles(k, nu), r)
+    return rq.Plan(D, r, U.astype(np.float32), V.astype(np.float32))
+
+
+def _line(workload: str, args, extra: dict) -> dict:
+    hbm_gbs, bf16_tf, src = peaks()
+    line = {"metric": METRIC, "workload": workload, "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "dtype": "bf16+int4", "data": "synthetic",
+            "peaks": {"hbm_gbs": hbm_gbs, "int8_tops": bf16_tf * INT8_OVER_BF16, "source": src}}
+    line.update(extra)
+    return line
+
+
+def run_workload(args):
+    """Workload configurations besides the headline step, one JSON line each."""
+    import numpy as np
+    import torch
+    import rotation_post_quantization_b200 as rq
+    import workloads as W
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    sptr = stream.cuda_stream
+    hbm_gbs, bf16_tf, _ = peaks()
+    int8_tops = bf16_tf * INT8_OVER_BF16
+    iters = max(3, args.steps)
+    g = torch.Generator(device=dev)
+    g.manual_seed(0)
+
+    def rand_codes(rows, K):
+        return torch.randint(0, 256, (rows, K // 2), generator=g, device=dev, dtype=torch.uint8)
+
+    def acts(N, D, w, seed):
+        return W.activations_bf16_fast(N, D, n_outlier=w.n_outlier, outlier_scale=w.outlier_scale,
+                                       dist=w.dist, seed=seed, device=str(dev))
+
+    name = args.workload
+    w = W.WORKLOADS[name]
+    if name == "tiny":
+        plan = _plan_for(rq, W, w.D, w.r, w.k, w.nu)
+        fx = W.workload_fixture(name)
+        x, res = fx.x.to(dev), fx.residual.to(dev)
+        h = torch.empty_like(x)
+        q = torch.empty(w.N, w.D // 2, dtype=torch.uint8, device=dev)
+        sc = torch.empty(w.N, dtype=torch.float32, device=dev)
+        f = lambda i: rq.respin_boundary_forward(plan, x, res, h, q, sc, sptr)
+        for i in range(args.warmup):
+            f(i)
+        us = _events_ms(torch, f, iters, stream) * 1e3
+        line = _line(name, args, {"config": {"D": w.D, "N": w.N, "r": w.r},
+                                  "boundary_us": us, "unit": "us", "value": us,
+                                  "higher_is_better": False,
+                                  "note": "latency of one boundary call (inputs L2-resident)"})
+    elif name == "decode":
+        plan = _plan_for(rq, W, w.D, w.r, w.k, w.nu)
+        NW = 16   # rotating weight sets: 16 x 8.4 MB > L2
+        wsets = [(rand_codes(w.O, w.D), torch.rand(w.O, generator=g, device=dev) * 1e-3 + 1e-3)
+                 for _ in range(NW)]
+        rows = []
+        for N in w.extra["Ns"]:
+            x, res = acts(N, w.D, w, 1), acts(N, w.D, w, 2)
+            h = torch.empty_like(x)
+            q = torch.empty(N, w.D // 2, dtype=torch.uint8, device=dev)
+            sc = torch.empty(N, dtype=torch.float32, device=dev)
+            out = torch.empty(N, w.O, dtype=torch.bfloat16, device=dev)
+            fb = lambda i: rq.respin_boundary_forward(plan, x, res, h, q, sc, sptr)
+            fg = lambda i: rq.w4a4_gemm(q, sc, wsets[i % NW][0], wsets[i % NW][1], out, sptr)
+            for i in range(args.warmup):
+                fb(i)
+                fg(i)
+            b_us = _events_ms(torch, fb, iters, stream) * 1e3
+            g_us = _events_ms(torch, fg, iters, stream) * 1e3
+            b_bytes = N * (6.5 * w.D + 4) + 2 * w.D * w.r * 2
+            g_bytes = w.O * w.D / 2 + N * w.D / 2 + N * w.O * 2 + 4 * (N + w.O)
+            rows.append({"N": N, "boundary_us": b_us, "gemm_us": g_us,
+                         "boundary_frac_of_hbm": b_bytes / hbm_gbs / 1e3 / b_us,
+                         "gemm_frac_of_hbm": g_bytes / hbm_gbs / 1e3 / g_us,
+                         "gemm_tops": 2.0 * N * w.D * w.O / g_us / 1e6})
+        line = _line(name, args, {"config": {"D": w.D, "r": w.r, "gemm": "%d -> %d" % (w.D, w.O),
+                                             "weights": "16 rotating sets (134 MB > L2)"},
+                                  "rows": rows, "unit": "us", "higher_is_better": False,
+                                  "note": "fractions: algorithmic bytes / HBM bandwidth / time"})
+    elif name == "llama2_70b":
+        N, D = w.N, w.D
+        sets = [(acts(N, D, w, 2 * i + 1), acts(N, D, w, 2 * i + 2)) for i in range(2)]
+        h = torch.empty(N, D, dtype=torch.bfloat16, device=dev)
+        q = torch.empty(N, D // 2, dtype=torch.uint8, device=dev)
+        sc = torch.empty(N, dtype=torch.float32, device=dev)
+        rows = []
+        for r in w.extra["ranks"]:
+            try:
+                plan = _plan_for(rq, W, D, r, w.k, w.nu)
+            except rq.RespinError as e:
+                rows.append({"r": r, "unsupported": str(e)})
+                continue
+            fb = lambda i: rq.respin_boundary_forward(plan, *sets[i % 2], h, q, sc, sptr)
+            for i in range(args.warmup):
+                fb(i)
+            b_us = _events_ms(torch, fb, iters, stream) * 1e3
+            b_bytes = N * (6.5 * D + 4) + 2 * D * r * 2
+            rows.append({"r": r, "boundary_us": b_us, "tokens_per_s": N / b_us * 1e6,
+                         "frac_of_hbm": b_bytes / hbm_gbs / 1e3 / b_us})
+            plan.destroy()
+        qw = rand_codes(w.O, D)
+        sw = torch.rand(w.O, generator=g, device=dev) * 1e-3 + 1e-3
+        out = torch.empty(N, w.O, dtype=torch.bfloat16, device=dev)
+        fg = lambda i: rq.w4a4_gemm(q, sc, qw, sw, out, sptr)
+        for i in range(args.warmup):
+            fg(i)
+        g_us = _events_ms(torch, fg, iters, stream) * 1e3
+        tops = 2.0 * N * D * w.O / g_us / 1e6
+        line = _line(name, args, {"config": {"D": D, "N": N, "gemm": "%d -> %d" % (D, w.O),
+                                             "dist": w.dist},
+                                  "boundary_rank_sweep": rows, "gemm_us": g_us, "gemm_tops": tops,
+                                  "gemm_frac_of_peak": tops / int8_tops,
+                                  "unit": "tokens/s", "higher_is_better": True})
+    else:   # llama3_8b_stack
+        N, D, M, L = w.N, w.D, w.extra["mlp"], w.extra["layers"]
+        plans = [_plan_for(rq, W, D, w.r, w.k, w.nu, seed=i) for i in range(2 * L)]
+        wup = [(rand_codes(M, D), torch.rand(M, generator=g, device=dev) * 1e-3 + 1e-3) for _ in range(L)]
+        wdn = [(rand_codes(D, M), torch.rand(D, generator=g, device=dev) * 1e-3 + 1e-3) for _ in range(L)]
+        xatt = [acts(N, D, w, 100 + i) for i in range(4)]
+        res0 = acts(N, D, w, 99)
+        resid = [torch.empty(N, D, dtype=torch.bfloat16, device=dev) for _ in range(2)]
+        q1 = torch.empty(N, D // 2, dtype=torch.uint8, device=dev)
+        s1 = torch.empty(N, dtype=torch.float32, device=dev)
+        u = torch.empty(N, M, dtype=torch.bfloat16, device=dev)
+        q2 = torch.empty(N, M // 2, dtype=torch.uint8, device=dev)
+        s2 = torch.empty(N, dtype=torch.float32, device=dev)
+        xm = torch.empty(N, D, dtype=torch.bfloat16, device=dev)
+        q3 = torch.empty(N, D // 2, dtype=torch.uint8, device=dev)
+        s3 = torch.empty(N, dtype=torch.float32, device=dev)
+        qonly = rq.Plan(M, 0)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(5 * L + 1)]
+
+        def stack(record):
+            # h1 -> resid[0], h2 -> resid[1]; the next layer reads resid[1]
+            cur = res0
+            for l in range(L):
+                h1 = resid[0]
+                if record: ev[5 * l].record(stream)
+                rq.respin_boundary_forward(plans[2 * l], xatt[l % 4], cur, h1, q1, s1, sptr)
+                if record: ev[5 * l + 1].record(stream)
+                rq.w4a4_gemm(q1, s1, wup[l][0], wup[l][1], u, sptr)
+                if record: ev[5 * l + 2].record(stream)
+                rq.respin_boundary_forward(qonly, u, None, None, q2, s2, sptr)
+                if record: ev[5 * l + 3].record(stream)
+                rq.w4a4_gemm(q2, s2, wdn[l][0], wdn[l][1], xm, sptr)
+                if record: ev[5 * l + 4].record(stream)
+                rq.respin_boundary_forward(plans[2 * l + 1], xm, h1, resid[1], q3, s3, sptr)
+                cur = resid[1]
+            if record: ev[5 * L].record(stream)
+
+        for _ in range(max(1, args.warmup // 5)):
+            stack(False)
+        torch.cuda.synchronize()
+        reps = max(1, min(args.steps, 5))
+        parts = np.zeros(5)
+        total = 0.0
+        for _ in range(reps):
+            stack(True)
+            torch.cuda.synchronize()
+            total += ev[0].elapsed_time(ev[5 * L])
+            for l in range(L):
+                for j in range(5):
+                    parts[j] += ev[5 * l + j].elapsed_time(ev[5 * l + j + 1])
+        ms = total / reps
+        parts = parts / reps / L * 1e3
+        ops = L * 2.0 * N * D * M * 2
+        line = _line(name, args, {"config": {"D": D, "N": N, "layers": L, "mlp": M, "r": w.r,
+                                             "chain": "attn boundary, GEMM D->mlp, quant-only mlp, "
+                                                      "GEMM mlp->D, mlp boundary (nonlinearity omitted)"},
+                                  "value": N / (ms * 1e-3), "unit": "tokens/s", "higher_is_better": True,
+                                  "ms_per_stack": ms,
+                                  "per_layer_us": {"attn_boundary": parts[0], "gemm_up": parts[1],
+                                                   "quant_only": parts[2], "gemm_down": parts[3],
+                                                   "mlp_boundary": parts[4]},
+                                  "gemm_tops": ops / ((parts[1] + parts[3]) * L * 1e-6) / 1e12,
+                                  "boundary_tokens_per_s": N / ((parts[0] + parts[4]) / 2 * 1e-6)})
+    if rq.respin_device_status() != 0:
+        raise RuntimeError("a kernel reported a device-side failure")
+    print(json.dumps(line), flush=True)
+
+
 def run_profile_launch(args):
     """Warm-up launches, then exactly one more launch of the chosen kernel."""
     import numpy as np
@@ -491,6 +699,9 @@ def main():
     rank, world, local_rank = rank_env()
     if args.impl == "reference":
         run_reference(args, rank)
+        return
+    if args.workload != "llama2_7b":
+        run_workload(args)
         return
     run_ours(args, rank, world, local_rank)
 

@@ -529,7 +529,9 @@ struct BoundarySmem {
   uint32_t us, vs, stage0, stage_bytes, partial, ybuf, wamax, am2, amaxbuf, rowinv, bars, total;
 };
 
-__host__ __device__ inline BoundarySmem boundary_smem_layout(int T, int R, int Dc) {
+// vres: V slice resident in shared memory (else read from global memory in
+// the re-projection).
+__host__ __device__ inline BoundarySmem boundary_smem_layout(int T, int R, int Dc, bool vres = true) {
   const int MT = T / 16, NT1 = R / 8;
   const int WN = (NT1 / 4) > 1 ? NT1 / 4 : 1;
   const int WK = 8 / (MT * WN);
@@ -538,7 +540,7 @@ __host__ __device__ inline BoundarySmem boundary_smem_layout(int T, int R, int D
   BoundarySmem L;
   uint32_t off = 0;
   L.us = off;          off += R * pitch;                          // U^T slice, padded rows
-  L.vs = off;          off += static_cast<uint32_t>(Dc) * R * 2;  // V slice, swizzled
+  L.vs = off;          off += vres ? static_cast<uint32_t>(Dc) * R * 2 : 0u;  // V slice, swizzled
   L.stage0 = off;      L.stage_bytes = 2 * T * pitch;  off += 2 * L.stage_bytes;
   L.partial = off;     off += WK * T * RP * 4;                    // y (padded) aliases [0]
   L.ybuf = off;        off += T * R * 4;
@@ -552,7 +554,9 @@ __host__ __device__ inline BoundarySmem boundary_smem_layout(int T, int R, int D
   return L;
 }
 
-template <int T, int R, bool F32OUT>
+// VRES = false: only the U^T slice is resident; the re-projection reads its V
+// fragments from global memory (L2), for shapes whose two slices do not fit.
+template <int T, int R, bool F32OUT, bool VRES = true>
 __global__ void __launch_bounds__(kBoundaryThreads, 1)
 boundary_cluster_smem_kernel(const bf16* __restrict__ x, const bf16* __restrict__ res,
                              const bf16* __restrict__ Ut,   // [R, D]  (U transposed, zero padded)
@@ -562,7 +566,7 @@ boundary_cluster_smem_kernel(const bf16* __restrict__ x, const bf16* __restrict_
   using C = SmemCfg<T, R>;
   constexpr int RP = C::RP;
   extern __shared__ __align__(128) uint8_t smem[];
-  const BoundarySmem L = boundary_smem_layout(T, R, Dc);
+  const BoundarySmem L = boundary_smem_layout(T, R, Dc, VRES);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, q4 = lane & 3;
   const uint32_t crank = cluster_ctarank();
@@ -599,7 +603,7 @@ boundary_cluster_smem_kernel(const bf16* __restrict__ x, const bf16* __restrict_
       const uint4 val = __ldg(reinterpret_cast<const uint4*>(Ut + static_cast<size_t>(n) * D + col0) + v);
       *reinterpret_cast<uint4*>(smem + L.us + n * pitch + v * 16) = val;
     }
-    for (int i = tid; i < Dc * C::CPR; i += kBoundaryThreads) {
+    for (int i = tid; VRES && i < Dc * C::CPR; i += kBoundaryThreads) {
       const int d = i / C::CPR, j = i % C::CPR;
       const uint4 val = __ldg(reinterpret_cast<const uint4*>(V + static_cast<size_t>(col0 + d) * R) + j);
       const int js = j ^ ((d / C::VL) & C::VXM);
@@ -704,7 +708,15 @@ boundary_cluster_smem_kernel(const bf16* __restrict__ x, const bf16* __restrict_
       for (int t8 = 0; t8 < ntw; ++t8) {
         const int d0 = (warp * ntw + t8) * 8;
         uint32_t b[C::KS2][2];
-        {
+        if constexpr (!VRES) {
+          // B fragment of column d0 + g: (V[d][16ks + 2q], +1) and (+8, +9)
+          const uint32_t* vr = reinterpret_cast<const uint32_t*>(V + static_cast<size_t>(col0 + d0 + g) * R) + q4;
+#pragma unroll
+          for (int ks = 0; ks < C::KS2; ++ks) {
+            b[ks][0] = __ldg(vr + 8 * ks);
+            b[ks][1] = __ldg(vr + 8 * ks + 4);
+          }
+        } else {
           const int d = d0 + (lane & 7);
           const uint32_t vrow = sbase + L.vs + d * (R * 2);
           const int sw = (d / C::VL) & C::VXM;

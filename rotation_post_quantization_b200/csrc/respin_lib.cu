@@ -156,17 +156,24 @@ size_t rowtile_smem(int R, int D) {
   return W == 16 ? RtCfg<32, 16>::smem(D) : RtCfg<32, 8>::smem(D);
 }
 
-template <int T, int R, bool F32>
+template <int T, int R, bool F32, bool VRES>
 const void* smem_fn() {
-  return reinterpret_cast<const void*>(&boundary_cluster_smem_kernel<T, R, F32>);
+  return reinterpret_cast<const void*>(&boundary_cluster_smem_kernel<T, R, F32, VRES>);
 }
 
-const void* pick_smem_fn(int T, int R, bool f32) {
+// vres = false: the V slice is read from global memory (16-token tiles,
+// r = 64 or 128 only).
+const void* pick_smem_fn(int T, int R, bool f32, bool vres) {
 #define RESPIN_PICK(TT, RR)                                                   \
-  if (T == TT && R == RR) return f32 ? smem_fn<TT, RR, true>() : smem_fn<TT, RR, false>();
-  RESPIN_PICK(32, 16) RESPIN_PICK(32, 32) RESPIN_PICK(32, 64)
-  RESPIN_PICK(16, 16) RESPIN_PICK(16, 32) RESPIN_PICK(16, 64) RESPIN_PICK(16, 128)
+  if (T == TT && R == RR) return f32 ? smem_fn<TT, RR, true, true>() : smem_fn<TT, RR, false, true>();
+  if (vres) {
+    RESPIN_PICK(32, 16) RESPIN_PICK(32, 32) RESPIN_PICK(32, 64)
+    RESPIN_PICK(16, 16) RESPIN_PICK(16, 32) RESPIN_PICK(16, 64) RESPIN_PICK(16, 128)
+    return nullptr;
+  }
 #undef RESPIN_PICK
+  if (T == 16 && R == 64) return f32 ? smem_fn<16, 64, true, false>() : smem_fn<16, 64, false, false>();
+  if (T == 16 && R == 128) return f32 ? smem_fn<16, 128, true, false>() : smem_fn<16, 128, false, false>();
   return nullptr;
 }
 
@@ -265,21 +272,24 @@ respin_status_t configure_boundary(int D, int R, bool f32, BoundaryConfig* out) 
       return ok();
     }
   }
-  for (int C : {1, 2, 4, 8, 16}) {
-    if (D % C) continue;
-    const int Dc = D / C;
-    if (Dc % 64) continue;
-    for (int T : {32, 16}) {
-      if (T * R > 2048) continue;
-      const void* fn = pick_smem_fn(T, R, f32);
-      if (!fn) continue;
-      const size_t smem = boundary_smem_layout(T, R, Dc).total;
-      if (smem > static_cast<size_t>(smem_optin)) continue;
-      const int n = max_active_clusters(fn, C, smem, kBoundaryThreads);
-      if (n <= 0) continue;
-      out->kind = kClusterSmem; out->rf = false; out->T = T; out->R = R; out->cluster = C; out->Dc = Dc;
-      out->smem = smem; out->max_clusters = n; out->fn = fn;
-      return ok();
+  // Shared-memory factor slices (both, else U^T only with V read from L2).
+  for (bool vres : {true, false}) {
+    for (int C : {1, 2, 4, 8, 16}) {
+      if (D % C) continue;
+      const int Dc = D / C;
+      if (Dc % 64) continue;
+      for (int T : {32, 16}) {
+        if (T * R > 2048) continue;
+        const void* fn = pick_smem_fn(T, R, f32, vres);
+        if (!fn) continue;
+        const size_t smem = boundary_smem_layout(T, R, Dc, vres).total;
+        if (smem > static_cast<size_t>(smem_optin)) continue;
+        const int n = max_active_clusters(fn, C, smem, kBoundaryThreads);
+        if (n <= 0) continue;
+        out->kind = kClusterSmem; out->rf = false; out->T = T; out->R = R; out->cluster = C; out->Dc = Dc;
+        out->smem = smem; out->max_clusters = n; out->fn = fn;
+        return ok();
+      }
     }
   }
   return fail(RESPIN_ERR_UNSUPPORTED,

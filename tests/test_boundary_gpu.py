@@ -31,6 +31,7 @@ CASES = [
     ("d8192_r32", 8192, 70, 32, 128, 0.1, 16, 100.0, "student_t3"),
     ("d8192_r64", 8192, 40, 64, 128, 0.1, 16, 100.0, "student_t3"),
     ("d1024_r128", 1024, 40, 128, 128, 0.5, 4, 50.0, "normal"),
+    ("d8192_r128", 8192, 24, 128, 128, 0.1, 16, 100.0, "student_t3"),
 ]
 
 
