@@ -78,9 +78,20 @@ struct respin_plan_s {
   int D = 0, r = 0, r_pad = 0;
   unsigned flags = 0;
   int device = -1;
-  __nv_bfloat16* factors = nullptr;  // 2 * D * r_pad bf16: U part then V part
+  __nv_bfloat16* factors = nullptr;  // 2 * D * r_pad bf16: U part then V part (layout of cfg)
   BoundaryConfig cfg;
+  // Second configuration for calls with few tokens (row-tile plans only: a
+  // cluster splits each tile over several SMs, so a short call is not one
+  // SM's whole chain), with its own factor layout.
+  bool has_small = false;
+  __nv_bfloat16* factors_small = nullptr;
+  BoundaryConfig cfg_small;
 };
+
+// Calls with at most this many tokens use cfg_small when the plan has one
+// (row tiles: one 16-token tile per SM; a 4-CTA cluster tile chain is about a
+// third as long, so clusters win until their tile rounds add up).
+constexpr int kSmallTokens = 1280;
 
 namespace {
 
@@ -236,7 +247,7 @@ int max_active_clusters(const void* fn, int C, size_t smem, int threads) {
 // Choose the boundary kernel. r <= 32: register-resident factors with 512
 // (else 256) columns per CTA. Otherwise: shared-memory factors, the smallest
 // cluster whose per-CTA slice fits, preferring 32-token tiles.
-respin_status_t configure_boundary(int D, int R, bool f32, BoundaryConfig* out) {
+respin_status_t configure_boundary(int D, int R, bool f32, BoundaryConfig* out, bool allow_rowtile = true) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
@@ -244,7 +255,7 @@ respin_status_t configure_boundary(int D, int R, bool f32, BoundaryConfig* out) 
   e = cudaDeviceGetAttribute(&smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
   // Whole 16-token rows per CTA, factors streamed from L2 (no cluster).
-  if (R <= 32 && (D == 1024 || D == 2048 || D == 4096)) {
+  if (allow_rowtile && R <= 32 && (D == 1024 || D == 2048 || D == 4096)) {
     const size_t smem = rowtile_smem(R, D);
     const void* fn = pick_rowtile_fn(R, D, f32);
     int sms = 0;
@@ -345,28 +356,51 @@ respin_status_t respin_plan_create(respin_plan_t* out, int D, int r, const float
         ub[static_cast<size_t>(d) * r_pad + j] = *reinterpret_cast<const uint16_t*>(&u);
         vb[static_cast<size_t>(d) * r_pad + j] = *reinterpret_cast<const uint16_t*>(&v);
       }
-    // Device layout: fragment order for the row-tile and the register-factor
+    // Device layouts: fragment order for the row-tile and the register-factor
     // kernels, else U^T [r_pad, D] followed by V [D, r_pad].
-    std::vector<uint32_t> dev_words(static_cast<size_t>(D) * r_pad, 0);  // 2 * D * r_pad bf16
-    if (p->cfg.kind == kRowTile) {
+    auto layout = [&](const BoundaryConfig& c) {
+      std::vector<uint32_t> w(static_cast<size_t>(D) * r_pad, 0);  // 2 * D * r_pad bf16
       const size_t half = static_cast<size_t>(D) * r_pad / 2;
-      rt_pack_factors(ub.data(), vb.data(), D, r_pad, dev_words.data(), dev_words.data() + half);
-    } else if (p->cfg.rf) {
-      const size_t half = static_cast<size_t>(D) * r_pad / 2;
-      rf_pack_factors(ub.data(), vb.data(), D, r_pad, p->cfg.T, p->cfg.Dc, dev_words.data(), dev_words.data() + half);
-    } else {
-      uint16_t* h16 = reinterpret_cast<uint16_t*>(dev_words.data());
-      for (int d = 0; d < D; ++d)
-        for (int j = 0; j < r_pad; ++j) {
-          h16[static_cast<size_t>(j) * D + d] = ub[static_cast<size_t>(d) * r_pad + j];
-          h16[static_cast<size_t>(r_pad) * D + static_cast<size_t>(d) * r_pad + j] =
-              vb[static_cast<size_t>(d) * r_pad + j];
-        }
+      if (c.kind == kRowTile) {
+        rt_pack_factors(ub.data(), vb.data(), D, r_pad, w.data(), w.data() + half);
+      } else if (c.rf) {
+        rf_pack_factors(ub.data(), vb.data(), D, r_pad, c.T, c.Dc, w.data(), w.data() + half);
+      } else {
+        uint16_t* h16 = reinterpret_cast<uint16_t*>(w.data());
+        for (int d = 0; d < D; ++d)
+          for (int j = 0; j < r_pad; ++j) {
+            h16[static_cast<size_t>(j) * D + d] = ub[static_cast<size_t>(d) * r_pad + j];
+            h16[static_cast<size_t>(r_pad) * D + static_cast<size_t>(d) * r_pad + j] =
+                vb[static_cast<size_t>(d) * r_pad + j];
+          }
+      }
+      return w;
+    };
+    auto upload = [&](const BoundaryConfig& c, __nv_bfloat16** dst) -> respin_status_t {
+      const std::vector<uint32_t> w = layout(c);
+      cudaError_t e2 = cudaMalloc(dst, w.size() * sizeof(uint32_t));
+      if (e2 != cudaSuccess) {
+        cudaGetLastError();
+        *dst = nullptr;
+        return fail(RESPIN_ERR_OOM, "cudaMalloc factors: %s", cudaGetErrorString(e2));
+      }
+      e2 = cudaMemcpy(*dst, w.data(), w.size() * sizeof(uint32_t), cudaMemcpyHostToDevice);
+      if (e2 != cudaSuccess) return cuda_fail(e2, "cudaMemcpy factors");
+      return ok();
+    };
+    respin_status_t st2 = upload(p->cfg, &p->factors);
+    if (st2 == RESPIN_OK && p->cfg.kind == kRowTile &&
+        configure_boundary(D, r_pad, (flags & RESPIN_H_FP32_DEBUG) != 0, &p->cfg_small, false) == RESPIN_OK) {
+      st2 = upload(p->cfg_small, &p->factors_small);
+      p->has_small = st2 == RESPIN_OK;
     }
-    e = cudaMalloc(&p->factors, dev_words.size() * sizeof(uint32_t));
-    if (e != cudaSuccess) { delete p; cudaGetLastError(); return fail(RESPIN_ERR_OOM, "cudaMalloc factors: %s", cudaGetErrorString(e)); }
-    e = cudaMemcpy(p->factors, dev_words.data(), dev_words.size() * sizeof(uint32_t), cudaMemcpyHostToDevice);
-    if (e != cudaSuccess) { cudaFree(p->factors); delete p; return cuda_fail(e, "cudaMemcpy factors"); }
+    t_last_error.clear();
+    if (st2 != RESPIN_OK || p->factors == nullptr) {
+      if (p->factors) cudaFree(p->factors);
+      if (p->factors_small) cudaFree(p->factors_small);
+      delete p;
+      return st2 != RESPIN_OK ? st2 : fail(RESPIN_ERR_OOM, "factor upload failed");
+    }
   }
   // The row kernels need the shared-memory carve-out only for their reduction.
   {
@@ -391,6 +425,7 @@ respin_status_t respin_plan_destroy(respin_plan_t plan) {
     cudaSetDevice(plan->device);
     cudaError_t e = cudaDeviceSynchronize();
     if (e == cudaSuccess) e = cudaFree(plan->factors);
+    if (e == cudaSuccess && plan->factors_small) e = cudaFree(plan->factors_small);
     if (e != cudaSuccess) st = cuda_fail(e, "releasing plan factors");
     cudaSetDevice(cur);
   }
@@ -436,14 +471,16 @@ respin_status_t respin_boundary_forward(respin_plan_t plan, const void* x, const
     return ok();
   }
 
-  const BoundaryConfig& c = plan->cfg;
+  const bool small = plan->has_small && N <= kSmallTokens;
+  const BoundaryConfig& c = small ? plan->cfg_small : plan->cfg;
+  const bf16* fac = small ? plan->factors_small : plan->factors;
   const int ntiles = (N + c.T - 1) / c.T;
   if (c.kind == kRowTile) {
     CUtensorMap tmR, tmX;
     if (!make_tmap_bf16_tile(&tmR, residual, N, D) || !make_tmap_bf16_tile(&tmX, x, N, D))
       return fail(RESPIN_ERR_CUDA, "cuTensorMapEncodeTiled failed for the boundary tiles");
-    const uint4* ut = reinterpret_cast<const uint4*>(plan->factors);
-    const uint4* vt = reinterpret_cast<const uint4*>(plan->factors + static_cast<size_t>(plan->r_pad) * D);
+    const uint4* ut = reinterpret_cast<const uint4*>(fac);
+    const uint4* vt = reinterpret_cast<const uint4*>(fac + static_cast<size_t>(plan->r_pad) * D);
     const int grid = ntiles < c.max_clusters ? ntiles : c.max_clusters;
     void* args[] = {&tmR, &tmX, &ut, &vt, &N, &h_out, &q_packed, &scale};
     cudaError_t e = cudaLaunchKernel(c.fn, dim3(grid), dim3(32 * c.cluster), args, c.smem, s);
@@ -465,13 +502,13 @@ respin_status_t respin_boundary_forward(respin_plan_t plan, const void* x, const
   lc.numAttrs = 1;
   cudaError_t e;
   if (c.rf) {
-    const uint4* uf = reinterpret_cast<const uint4*>(plan->factors);
-    const uint4* vf = reinterpret_cast<const uint4*>(plan->factors + static_cast<size_t>(plan->r_pad) * D);
+    const uint4* uf = reinterpret_cast<const uint4*>(fac);
+    const uint4* vf = reinterpret_cast<const uint4*>(fac + static_cast<size_t>(plan->r_pad) * D);
     void* args[] = {&xb, &rb, &uf, &vf, &N, const_cast<int*>(&D), &h_out, &q_packed, &scale};
     e = cudaLaunchKernelExC(&lc, c.fn, args);
   } else {
-    const bf16* ut = plan->factors;
-    const bf16* v = plan->factors + static_cast<size_t>(plan->r_pad) * D;
+    const bf16* ut = fac;
+    const bf16* v = fac + static_cast<size_t>(plan->r_pad) * D;
     int Dc = c.Dc;
     void* args[] = {&xb, &rb, &ut, &v, &N, const_cast<int*>(&D), &Dc, &h_out, &q_packed, &scale};
     e = cudaLaunchKernelExC(&lc, c.fn, args);

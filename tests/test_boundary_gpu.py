@@ -32,6 +32,10 @@ CASES = [
     ("d8192_r64", 8192, 40, 64, 128, 0.1, 16, 100.0, "student_t3"),
     ("d1024_r128", 1024, 40, 128, 128, 0.5, 4, 50.0, "normal"),
     ("d8192_r128", 8192, 24, 128, 128, 0.1, 16, 100.0, "student_t3"),
+    # above the small-call threshold: row-tile kernel (16 whole tokens per CTA)
+    ("rowtile_d4096_ragged", 4096, 1301, 32, 64, 0.1, 8, 50.0, "normal"),
+    ("rowtile_d4096_nu1", 4096, 1296, 32, 64, 1.0, 8, 50.0, "normal"),
+    ("rowtile_d2048_r16", 2048, 1290, 16, 32, 0.5, 4, 20.0, "student_t3"),
 ]
 
 
