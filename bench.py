@@ -156,9 +156,23 @@ def oracle_sample_rate(fx, qw, sw, n_boundary: int, n_gemm: int):
     return 1.0 / per_tok, (t2 - t0)
 
 
+def host_cpu() -> str:
+    """CPU model of the host (the oracle's machine) and its logical core count."""
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as fh:
+            for line in fh:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return "%s, %d logical cores" % (model, os.cpu_count() or 0)
+
+
 def cpu_baseline_block(fx, qw, sw):
     rate, secs = oracle_sample_rate(fx, qw, sw, 2048, 160)
-    return {"value": rate, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+    return {"value": rate, "unit": "tokens/s", "cores": 1, "kind": "oracle", "cpu": host_cpu(),
             "sample": "boundary oracle (fp64 fix + binary32 quantizer) on all "
                       "2048 tokens, W4A4 GEMM oracle (exact int64 + binary32 "
                       "epilogue) on 160 of the 2048 rows x 11008 channels; "
@@ -202,7 +216,7 @@ def run_reference(args, rank: int):
         "dtype": "f64+f32+int64", "data": "synthetic",
         "config": config_block(w, args.gpus),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1,
-                         "kind": "oracle",
+                         "kind": "oracle", "cpu": host_cpu(),
                          "sample": "each step: boundary oracle on 64 tokens "
                                    "+ GEMM oracle on 4 rows, 1 thread; "
                                    "%.1f s total" % t},
