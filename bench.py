@@ -483,6 +483,31 @@ def _events_ms(torch, fn, iters: int, stream) -> float:
     return e0.elapsed_time(e1) / iters
 
 
+def _graph_ms(torch, fn, iters: int) -> float:
+    """Mean device time per call of fn(i) captured `iters` times in one CUDA
+    graph and replayed (no host launch overhead between the calls)."""
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        for i in range(3):
+            fn(i)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=side):
+        for i in range(iters):
+            fn(i)
+    graph.replay()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    graph.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    del graph
+    return e0.elapsed_time(e1) / iters
+
+
 def _plan_for(rq, W, D, r, k, nu, seed=0):
     import numpy as np
     Q = W.orthonormal_basis(D, k, seed)
@@ -552,23 +577,29 @@ def run_workload(args):
             q = torch.empty(N, w.D // 2, dtype=torch.uint8, device=dev)
             sc = torch.empty(N, dtype=torch.float32, device=dev)
             out = torch.empty(N, w.O, dtype=torch.bfloat16, device=dev)
-            fb = lambda i: rq.respin_boundary_forward(plan, x, res, h, q, sc, sptr)
-            fg = lambda i: rq.w4a4_gemm(q, sc, wsets[i % NW][0], wsets[i % NW][1], out, sptr)
+            # the current stream: the graph's capture stream inside _graph_ms
+            fb = lambda i: rq.respin_boundary_forward(plan, x, res, h, q, sc)
+            fg = lambda i: rq.w4a4_gemm(q, sc, wsets[i % NW][0], wsets[i % NW][1], out)
             for i in range(args.warmup):
                 fb(i)
                 fg(i)
-            b_us = _events_ms(torch, fb, iters, stream) * 1e3
-            g_us = _events_ms(torch, fg, iters, stream) * 1e3
+            eb_us = _events_ms(torch, fb, iters, stream) * 1e3
+            eg_us = _events_ms(torch, fg, iters, stream) * 1e3
+            b_us = _graph_ms(torch, fb, iters) * 1e3
+            g_us = _graph_ms(torch, fg, iters) * 1e3
             b_bytes = N * (6.5 * w.D + 4) + 2 * w.D * w.r * 2
             g_bytes = w.O * w.D / 2 + N * w.D / 2 + N * w.O * 2 + 4 * (N + w.O)
             rows.append({"N": N, "boundary_us": b_us, "gemm_us": g_us,
+                         "eager_boundary_us": eb_us, "eager_gemm_us": eg_us,
                          "boundary_frac_of_hbm": b_bytes / hbm_gbs / 1e3 / b_us,
                          "gemm_frac_of_hbm": g_bytes / hbm_gbs / 1e3 / g_us,
                          "gemm_tops": 2.0 * N * w.D * w.O / g_us / 1e6})
         line = _line(name, args, {"config": {"D": w.D, "r": w.r, "gemm": "%d -> %d" % (w.D, w.O),
                                              "weights": "16 rotating sets (134 MB > L2)"},
                                   "rows": rows, "unit": "us", "higher_is_better": False,
-                                  "note": "fractions: algorithmic bytes / HBM bandwidth / time"})
+                                  "note": "times: CUDA-graph replay (device time per call); eager_*: "
+                                          "back-to-back calls from Python (host-bound at these sizes). "
+                                          "fractions: algorithmic bytes / HBM bandwidth / graph time"})
     elif name == "llama2_70b":
         N, D = w.N, w.D
         sets = [(acts(N, D, w, 2 * i + 1), acts(N, D, w, 2 * i + 2)) for i in range(2)]

@@ -45,6 +45,13 @@
 //    every SM widens and stores half the weight bytes it would alone;
 //  * 4 epilogue warps drain the other TMEM buffer (tcgen05.ld), apply the two
 //    scales and store bf16, overlapping the next tile's main loop.
+// Split K (SPLIT > 1, single CTAs, few tiles - e.g. decode): a cluster of
+// SPLIT CTAs computes one tile, CTA k over K blocks [k KB/S, (k+1) KB/S).
+// After a cluster barrier (every CTA's MMAs are done, so the widened and
+// packed stage rings, contiguous from the base, are free) each CTA writes its
+// partial int32 accumulators of the columns that CTA j owns (256/S of them)
+// into CTA j's rings with distributed-shared-memory stores; after a second barrier CTA j sums the S partials in rank order
+// (exact, deterministic) and runs the usual epilogue on its columns.
 #pragma once
 
 #include <cuda.h>
@@ -66,10 +73,10 @@ constexpr int kGemmTmaWarp = kGemmEpiWarp0 + kGemmEpilogueWarps;  // warp 13
 constexpr int kGemmThreads = (kGemmTmaWarp + 1) * 32;
 
 #ifndef RESPIN_GEMM_US1
-#define RESPIN_GEMM_US1 3
+#define RESPIN_GEMM_US1 2
 #endif
 #ifndef RESPIN_GEMM_PS1
-#define RESPIN_GEMM_PS1 2
+#define RESPIN_GEMM_PS1 4
 #endif
 #ifndef RESPIN_GEMM_EB
 #define RESPIN_GEMM_EB 2
@@ -123,12 +130,15 @@ __device__ __forceinline__ uint32_t sw64_offset(int r, int j) {
 // (inner dimension first), no swizzle, out-of-range elements zero filled.
 // tmO: the output [N, O] (bf16, or int32 for I32OUT), box {64 bytes, 32 rows},
 // 64-byte swizzle; the store clips rows >= N and columns >= O.
-template <int CG, bool I32OUT>
+template <int CG, bool I32OUT, int SPLIT = 1>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const __grid_constant__ CUtensorMap tmO, const float* __restrict__ sa,
                  const float* __restrict__ sw, int N, int K, int O) {
   using G = GemmCfg<CG>;
+  static_assert(SPLIT == 1 || CG == 1, "split K runs on single CTAs");
+  static_assert(SPLIT == 1 || SPLIT * (kGemmBM * kGemmBN * 4 / SPLIT) <= G::US * G::Stage + G::PS * G::PStage,
+                "split-K receive slots fit in the (idle) stage rings");
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -147,9 +157,13 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t rank = CG == 2 ? cluster_ctarank() : 0u;
-  const int group = CG == 2 ? static_cast<int>(blockIdx.x) / 2 : static_cast<int>(blockIdx.x);
-  const int ngroups = CG == 2 ? static_cast<int>(gridDim.x) / 2 : static_cast<int>(gridDim.x);
-  const int KB = K / kGemmBK;
+  constexpr int CL = CG * SPLIT;   // CTAs per cluster
+  const int group = static_cast<int>(blockIdx.x) / CL;
+  const int ngroups = static_cast<int>(gridDim.x) / CL;
+  // K blocks of this CTA: all of them, or its share of a split-K cluster
+  const uint32_t krank = SPLIT > 1 ? cluster_ctarank() : 0u;
+  const int KB = K / kGemmBK / SPLIT;
+  const int kb0 = static_cast<int>(krank) * KB;
   const int mtiles = (N + G::TileM - 1) / G::TileM;
   const int ntiles = (O + kGemmBN - 1) / kGemmBN;
   const int tiles = mtiles * ntiles;
@@ -186,11 +200,76 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   const uint32_t full_leader0 = CG == 2 ? map_to_rank(full0, 0) : full0;
   const uint32_t aempty_leader0 = CG == 2 ? map_to_rank(aempty0, 0) : aempty0;
 
+  // Epilogue output staging (epilogue warps): EB 32 x 64-byte units per warp,
+  // each written to global memory by one tensor store.
+  const int quad = warp & 3;   // hardware rule: warp w reads TMEM lanes 32*(w%4)..
+  const uint32_t ubase = ebase + static_cast<uint32_t>(quad * G::EB * G::Unit);
+  int unit = 0;
+  auto stage_unit = [&](const uint4 (&piece)[4], int x, int y) {
+    if (lane == 0) bulk_wait_group_read<G::EB - 1>();   // this unit's previous store read it
+    __syncwarp();
+    const uint32_t u = ubase + static_cast<uint32_t>((unit % G::EB) * G::Unit);
+    uint8_t* up = smem + (u - base);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) *reinterpret_cast<uint4*>(up + sw64_offset(lane, j)) = piece[j];
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_2d(&tmO, x, y, u);
+      bulk_commit_group();
+    }
+    ++unit;
+  };
+  // One 32-column chunk of accumulators (256 acc each, lane = row `row` of the
+  // tile) -> scaled bf16 (or int32) output block at (colb, y) via staging.
+  auto store_chunk = [&](const uint32_t (&v)[32], int colb, int y, float sa_r, const float* swp) {
+    if constexpr (I32OUT) {
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        if (colb + 16 * half >= O) break;
+        uint4 piece[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int e = 16 * half + 4 * j;
+          piece[j] = make_uint4(static_cast<uint32_t>(static_cast<int32_t>(v[e]) >> 8),
+                                static_cast<uint32_t>(static_cast<int32_t>(v[e + 1]) >> 8),
+                                static_cast<uint32_t>(static_cast<int32_t>(v[e + 2]) >> 8),
+                                static_cast<uint32_t>(static_cast<int32_t>(v[e + 3]) >> 8));
+        }
+        stage_unit(piece, colb + 16 * half, y);
+      }
+    } else {
+      uint4 piece[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (colb + 8 * j >= O) {   // O % 16 == 0: a chunk is full or half full
+          piece[j] = make_uint4(0u, 0u, 0u, 0u);
+          continue;
+        }
+        const float4 w0 = reinterpret_cast<const float4*>(swp)[2 * j];
+        const float4 w1 = reinterpret_cast<const float4*>(swp)[2 * j + 1];
+        const float ws[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+        uint32_t w[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int e = 8 * j + 2 * u;
+          const float f0 = __fmul_rn(__fmul_rn(exact_i22_to_f32(static_cast<int32_t>(v[e]) >> 8), sa_r), ws[2 * u]);
+          const float f1 =
+              __fmul_rn(__fmul_rn(exact_i22_to_f32(static_cast<int32_t>(v[e + 1]) >> 8), sa_r), ws[2 * u + 1]);
+          w[u] = pack_bf16x2(f0, f1);
+        }
+        piece[j] = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+      stage_unit(piece, colb, y);
+    }
+  };
+
   if (warp < kGemmProducerWarps) {
     // ------------------------------------------------ producers: widen packed -> int8
     bool ok = true;
     int kstep = 0;  // running k-block counter over all tiles (selects the stages)
     for (int t = group; t < tiles; t += ngroups) {
+      const int m_base = (t / ntiles) * G::TileM + static_cast<int>(rank) * kGemmBM;
       for (int kb = 0; kb < KB; ++kb, ++kstep) {
         const int ps = kstep % G::PS, s = kstep % G::US;
         if (ok) ok = mbar_wait(pfull0 + 8 * ps, (kstep / G::PS) & 1, kSiteGemmPackedFull);
@@ -207,6 +286,10 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
           const bool is_a = q < kGemmBM * 4;
           const int qq = is_a ? q : q - kGemmBM * 4;
           const int row = qq >> 2, c = qq & 3;
+          // A rows past N: the accumulator rows they feed are never stored,
+          // so whatever the stage holds there is fine (saves the widening of
+          // mostly empty A tiles at small N)
+          if (is_a && m_base + row >= N) continue;
           uint8_t* rowp = sA + (is_a ? 0 : G::AStage) + (row >> 3) * 1024 + (row & 7) * 128;
           const uint4 p = b[j];
           const uint4 lo = make_uint4((p.x << 4) & 0xF0F0F0F0u, (p.y << 4) & 0xF0F0F0F0u,
@@ -249,8 +332,8 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
           if (!ok) continue;
           const uint32_t dst = pbase + ps * G::PStage;
           mbar_arrive_expect_tx(pfull0 + 8 * ps, bytes);
-          if (is_b) tma_load_2d(dst + G::PAStage, &tmB, kb * (kGemmBK / 2), brow, pfull0 + 8 * ps);
-          else tma_load_2d(dst, &tmA, kb * (kGemmBK / 2), arow, pfull0 + 8 * ps);
+          if (is_b) tma_load_2d(dst + G::PAStage, &tmB, (kb0 + kb) * (kGemmBK / 2), brow, pfull0 + 8 * ps);
+          else tma_load_2d(dst, &tmA, (kb0 + kb) * (kGemmBK / 2), arow, pfull0 + 8 * ps);
         }
       }
     }
@@ -300,27 +383,10 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     // lane issues a TMA tensor store of the 32 x 32 block, so every output
     // row segment reaches L2 as whole sectors. int32 output takes two units
     // (16 columns each) per chunk.
-    const int quad = warp & 3;   // hardware rule: warp w reads TMEM lanes 32*(w%4)..
-    const uint32_t ubase = ebase + static_cast<uint32_t>(quad * G::EB * G::Unit);
     float* sws = reinterpret_cast<float*>(smem + (swbase - base) + quad * G::SwBytes);
     bool ok = true;
-    int local = 0, unit = 0;
-    auto stage_unit = [&](const uint4 (&piece)[4], int x, int y) {
-      if (lane == 0) bulk_wait_group_read<G::EB - 1>();   // this unit's previous store read it
-      __syncwarp();
-      const uint32_t u = ubase + static_cast<uint32_t>((unit % G::EB) * G::Unit);
-      uint8_t* up = smem + (u - base);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) *reinterpret_cast<uint4*>(up + sw64_offset(lane, j)) = piece[j];
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) {
-        tma_store_2d(&tmO, x, y, u);
-        bulk_commit_group();
-      }
-      ++unit;
-    };
-    for (int t = group; t < tiles; t += ngroups, ++local) {
+    int local = 0;
+    for (int t = group; SPLIT == 1 && t < tiles; t += ngroups, ++local) {
       const int ab = local & 1;
       const int m0 = (t / ntiles) * G::TileM + static_cast<int>(rank) * kGemmBM;
       const int n0 = (t % ntiles) * kGemmBN;
@@ -357,46 +423,7 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         for (int h = 0; h < 2; ++h) {
           const int colb = n0 + (cc + h) * 32;
           if (colb >= O) break;
-          if constexpr (I32OUT) {
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-              if (colb + 16 * half >= O) break;
-              uint4 piece[4];
-#pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                const int e = 16 * half + 4 * j;
-                piece[j] = make_uint4(static_cast<uint32_t>(static_cast<int32_t>(v[h][e]) >> 8),
-                                      static_cast<uint32_t>(static_cast<int32_t>(v[h][e + 1]) >> 8),
-                                      static_cast<uint32_t>(static_cast<int32_t>(v[h][e + 2]) >> 8),
-                                      static_cast<uint32_t>(static_cast<int32_t>(v[h][e + 3]) >> 8));
-              }
-              stage_unit(piece, colb + 16 * half, y);
-            }
-          } else {
-            uint4 piece[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              if (colb + 8 * j >= O) {   // O % 16 == 0: a chunk is full or half full
-                piece[j] = make_uint4(0u, 0u, 0u, 0u);
-                continue;
-              }
-              const float4 w0 = reinterpret_cast<const float4*>(sws)[(colb - n0) / 4 + 2 * j];
-              const float4 w1 = reinterpret_cast<const float4*>(sws)[(colb - n0) / 4 + 2 * j + 1];
-              const float ws[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-              uint32_t w[4];
-#pragma unroll
-              for (int u = 0; u < 4; ++u) {
-                const int e = 8 * j + 2 * u;
-                const float f0 = __fmul_rn(
-                    __fmul_rn(exact_i22_to_f32(static_cast<int32_t>(v[h][e]) >> 8), sa_r), ws[2 * u]);
-                const float f1 = __fmul_rn(
-                    __fmul_rn(exact_i22_to_f32(static_cast<int32_t>(v[h][e + 1]) >> 8), sa_r), ws[2 * u + 1]);
-                w[u] = pack_bf16x2(f0, f1);
-              }
-              piece[j] = make_uint4(w[0], w[1], w[2], w[3]);
-            }
-            stage_unit(piece, colb, y);
-          }
+          store_chunk(v[h], colb, y, sa_r, sws + (colb - n0));
         }
       }
       // hand the accumulator buffer back to the MMA warp (of the leader CTA)
@@ -407,9 +434,70 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         else mbar_arrive(aempty0 + 8 * ab);
       }
     }
+    if constexpr (SPLIT > 1) {
+      // one tile per cluster: its accumulators, then the reduction below
+      if (group < tiles && ok) ok = mbar_wait(afull0, 0, kSiteGemmAccum);
+    }
     // the staging units must not be released while a store still reads them
     if (lane == 0) bulk_wait_group_all();
     __syncwarp();
+  }
+  if constexpr (SPLIT > 1) {
+    // ---------------------------------------------- split-K reduction
+    constexpr int OC = kGemmBN / SPLIT;          // columns each CTA finishes
+    constexpr int SLOT = kGemmBM * OC * 4;       // one partial: 128 rows x OC int32
+    const bool live = group < tiles;
+    const int m0 = (group / ntiles) * G::TileM, n0 = (group % ntiles) * kGemmBN;
+    const int row = quad * 32 + lane;
+    // 16-byte piece pi of a row slot stored at (pi & ~7) | ((pi ^ row) & 7):
+    // the 32 lanes of a warp (32 rows) spread over 8 bank groups
+    auto pos16 = [&](int pi) { return ((pi & ~7) | ((pi ^ row) & 7)) * 16; };
+    tc_fence_before();
+    cluster_sync();   // every CTA's MMAs are done: its stage ring may be overwritten
+    if (warp >= kGemmEpiWarp0 && live) {
+      tc_fence_after();
+      const uint32_t tb = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+#pragma unroll 1
+      for (int cc = 0; cc < kGemmBN / 32; ++cc) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tb + cc * 32, v);
+        tmem_wait_ld();
+        const uint32_t owner = static_cast<uint32_t>(cc * 32 / OC);
+        const int p0 = (cc * 32 % OC) / 4;       // first 16-byte piece in the owner's row slot
+        if (m0 + row >= N) continue;   // rows past N are never stored: not sent either
+        const uint32_t dst = map_to_rank(base + krank * SLOT + row * (OC * 4), owner);
+#pragma unroll
+        for (int p = 0; p < 8; ++p)
+          st_dsmem_u32x4(dst + pos16(p0 + p), make_uint4(v[4 * p], v[4 * p + 1], v[4 * p + 2], v[4 * p + 3]));
+      }
+    }
+    cluster_sync();   // all partials delivered
+    if (warp >= kGemmEpiWarp0 && live) {
+      const int y = m0 + quad * 32;
+      const float sa_r = (!I32OUT && m0 + row < N) ? __ldg(sa + m0 + row) : 0.f;
+#pragma unroll 1
+      for (int cg = 0; cg < OC / 32; ++cg) {
+        uint32_t v[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) v[e] = 0u;
+        for (int sl = 0; m0 + row < N && sl < SPLIT; ++sl) {   // rank order: the same sum on every call
+          const uint8_t* src = smem + sl * SLOT + row * (OC * 4);
+#pragma unroll
+          for (int p = 0; p < 8; ++p) {
+            const uint4 w = *reinterpret_cast<const uint4*>(src + pos16(cg * 8 + p));
+            v[4 * p] += w.x;
+            v[4 * p + 1] += w.y;
+            v[4 * p + 2] += w.z;
+            v[4 * p + 3] += w.w;
+          }
+        }
+        const int colb = n0 + static_cast<int>(krank) * OC + cg * 32;
+        if (colb >= O || y >= N) continue;
+        store_chunk(v, colb, y, sa_r, I32OUT ? nullptr : sw + colb);   // channel scales read from global
+      }
+      if (lane == 0) bulk_wait_group_all();
+      __syncwarp();
+    }
   }
   tc_fence_before();
   // Neither CTA of a pair may release its TMEM or shared memory while the
