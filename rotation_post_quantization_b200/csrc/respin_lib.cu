@@ -144,28 +144,22 @@ const void* rowtile_fn() {
   return reinterpret_cast<const void*>(&boundary_rowtile_kernel<R, W, NB, F32>);
 }
 
-// Warps per CTA of the row-tile kernel for a given D (16 where D / 16 still
-// holds whole 64-column blocks, for more latency hiding per SM).
-#ifndef RESPIN_RT_WARPS
-#define RESPIN_RT_WARPS 8
-#endif
-int rowtile_warps(int D) { return RESPIN_RT_WARPS == 16 && D >= 2048 ? 16 : 8; }
+// Warps per CTA of the row-tile kernel (8: the register budget of the
+// prefetched factor fragments; 16 warps with shallower prefetch measured
+// slower).
+int rowtile_warps(int) { return 8; }
 
 const void* pick_rowtile_fn(int R, int D, bool f32) {
-  const int W = rowtile_warps(D), NB = D / (64 * W);
-#define RESPIN_PICK(RR, WW, BB) \
-  if (R == RR && W == WW && NB == BB) return f32 ? rowtile_fn<RR, WW, BB, true>() : rowtile_fn<RR, WW, BB, false>();
-  RESPIN_PICK(16, 8, 2) RESPIN_PICK(16, 8, 4) RESPIN_PICK(16, 8, 8) RESPIN_PICK(16, 16, 2) RESPIN_PICK(16, 16, 4)
-  RESPIN_PICK(32, 8, 2) RESPIN_PICK(32, 8, 4) RESPIN_PICK(32, 8, 8) RESPIN_PICK(32, 16, 2) RESPIN_PICK(32, 16, 4)
+  const int NB = D / (64 * 8);
+#define RESPIN_PICK(RR, BB) \
+  if (R == RR && NB == BB) return f32 ? rowtile_fn<RR, 8, BB, true>() : rowtile_fn<RR, 8, BB, false>();
+  RESPIN_PICK(16, 2) RESPIN_PICK(16, 4) RESPIN_PICK(16, 8)
+  RESPIN_PICK(32, 2) RESPIN_PICK(32, 4) RESPIN_PICK(32, 8)
 #undef RESPIN_PICK
   return nullptr;
 }
 
-size_t rowtile_smem(int R, int D) {
-  const int W = rowtile_warps(D);
-  if (R == 16) return W == 16 ? RtCfg<16, 16>::smem(D) : RtCfg<16, 8>::smem(D);
-  return W == 16 ? RtCfg<32, 16>::smem(D) : RtCfg<32, 8>::smem(D);
-}
+size_t rowtile_smem(int R, int D) { return R == 16 ? RtCfg<16, 8>::smem(D) : RtCfg<32, 8>::smem(D); }
 
 template <int T, int R, bool F32, bool VRES>
 const void* smem_fn() {
