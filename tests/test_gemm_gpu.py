@@ -58,6 +58,11 @@ def check(qa, qw, sa, sw, acc, outb, rows=None):
     (200, 1024, 272),      # ragged M and N tiles, several K blocks
     (300, 4096, 512),
     (64, 14336, 4096),     # down-projection K (stack workload)
+    # split K over clusters of single CTAs (few tiles)
+    (16, 1024, 4096),      # split 2 (8 K blocks)
+    (33, 4096, 4112),      # split 4; last tile 16 channels wide, ragged rows
+    (128, 2048, 272),      # split 4; owners of columns past O idle, full A tile
+    (3, 8192, 1040),       # split 4, 64 K blocks, 5 tiles
 ])
 def test_gemm_small(N, K, O_):
     qa, qw, sa, sw = make(N, K, O_)
