@@ -308,17 +308,27 @@ boundary_rowtile_kernel(const __grid_constant__ CUtensorMap tmR, const __grid_co
           mma_bf16_16816(acc[t], alo[kk], u4c(v, ri % 4), u4c(v, ri % 4 + 1));
         }
       }
+      // All loads of the block first, then the arithmetic, then the stores:
+      // h' overwrites the residual in place at XOR-computed offsets, which
+      // the compiler cannot prove distinct, so interleaved loads and stores
+      // would serialise the 16 pairs of a lane into one dependency chain.
+      uint32_t rw[8][2], xw[8][2];
+#pragma unroll
+      for (int t = 0; t < 8; ++t)
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const uint32_t off = rb[hh] ^ static_cast<uint32_t>(t << 4);
+          rw[t][hh] = *reinterpret_cast<const uint32_t*>(blk + off);
+          xw[t][hh] = *reinterpret_cast<const uint32_t*>(xblk + off);
+        }
 #pragma unroll
       for (int t = 0; t < 8; ++t) {
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
-          const uint32_t off = rb[hh] ^ static_cast<uint32_t>(t << 4);
-          const uint32_t rw = *reinterpret_cast<const uint32_t*>(blk + off);
-          const uint32_t xw = *reinterpret_cast<const uint32_t*>(xblk + off);
-          const float2 sum = add_f32x2(bf16x2_to_f32x2(rw), bf16x2_to_f32x2(xw));
+          const float2 sum = add_f32x2(bf16x2_to_f32x2(rw[t][hh]), bf16x2_to_f32x2(xw[t][hh]));
           const float2 h = add_f32x2(sum, make_float2(acc[t][2 * hh], acc[t][2 * hh + 1]));
           const uint32_t hb = pack_bf16x2(h.x, h.y);
-          *reinterpret_cast<uint32_t*>(blk + off) = hb;
+          rw[t][hh] = hb;
           amax2[hh] = absmax_bf16x2(amax2[hh], hb);
           if constexpr (F32OUT) {
             const int row = g + 8 * hh;
@@ -328,6 +338,11 @@ boundary_rowtile_kernel(const __grid_constant__ CUtensorMap tmR, const __grid_co
           }
         }
       }
+#pragma unroll
+      for (int t = 0; t < 8; ++t)
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh)
+          *reinterpret_cast<uint32_t*>(blk + (rb[hh] ^ static_cast<uint32_t>(t << 4))) = rw[t][hh];
       // the slot's bytes were read (generic proxy) before its next tensor copy
       fence_proxy_async_smem();
       __syncwarp();
