@@ -398,18 +398,33 @@ boundary_cluster_rf_kernel(const bf16* __restrict__ x, const bf16* __restrict__ 
       __nv_bfloat162 rmax2[C::MT];   // .x: row mt*16+g, .y: row mt*16+g+8
 #pragma unroll
       for (int mt = 0; mt < C::MT; ++mt) rmax2[mt] = __float2bfloat162_rn(0.f);
+      // The residual/x words of the next n8 tile are loaded before this
+      // tile's h' is stored in place: the compiler cannot tell the
+      // computed offsets apart, so loads after a store would wait for it.
+      auto load_rx = [&](int t, int mt, uint32_t (&w)[4]) {
+        const uint32_t offA = (mt * 16 + g) * pitch + ((warp * C::NTW + t) * 8 + 2 * q4) * 2;
+        w[0] = *reinterpret_cast<const uint32_t*>(rs_ptr + offA);
+        w[1] = *reinterpret_cast<const uint32_t*>(xs_ptr + offA);
+        w[2] = *reinterpret_cast<const uint32_t*>(rs_ptr + offA + 8 * pitch);
+        w[3] = *reinterpret_cast<const uint32_t*>(xs_ptr + offA + 8 * pitch);
+      };
+      uint32_t rx[2][C::MT][4];
+#pragma unroll
+      for (int mt = 0; mt < C::MT; ++mt) load_rx(0, mt, rx[0][mt]);
 #pragma unroll
       for (int t = 0; t < C::NTW; ++t) {
         const int d0 = (warp * C::NTW + t) * 8;
+        if (t + 1 < C::NTW) {
+#pragma unroll
+          for (int mt = 0; mt < C::MT; ++mt) load_rx(t + 1, mt, rx[(t + 1) & 1][mt]);
+        }
 #pragma unroll
         for (int mt = 0; mt < C::MT; ++mt) {
           const int rowA = mt * 16 + g;
           const uint32_t offA = rowA * pitch + (d0 + 2 * q4) * 2;
           const uint32_t offB = offA + 8 * pitch;
-          const uint32_t rA = *reinterpret_cast<const uint32_t*>(rs_ptr + offA);
-          const uint32_t xA = *reinterpret_cast<const uint32_t*>(xs_ptr + offA);
-          const uint32_t rB = *reinterpret_cast<const uint32_t*>(rs_ptr + offB);
-          const uint32_t xB = *reinterpret_cast<const uint32_t*>(xs_ptr + offB);
+          const uint32_t rA = rx[t & 1][mt][0], xA = rx[t & 1][mt][1];
+          const uint32_t rB = rx[t & 1][mt][2], xB = rx[t & 1][mt][3];
           // accumulators start at residual + x; the tensor cores add y V^T
           float acc[4] = {bf16_lo_f32(rA) + bf16_lo_f32(xA), bf16_hi_f32(rA) + bf16_hi_f32(xA),
                           bf16_lo_f32(rB) + bf16_lo_f32(xB), bf16_hi_f32(rB) + bf16_hi_f32(xB)};
