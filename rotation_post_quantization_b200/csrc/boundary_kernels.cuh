@@ -101,19 +101,34 @@ __device__ __forceinline__ void stage_tile(const bf16* __restrict__ x, const bf1
   }
 }
 
+// Residual and x words (bf16 pairs at column `colc`) of rows g and g + 8 of
+// every m16 tile, read before the previous n8 block's in-place stores so the
+// loads need not wait behind them.
+template <int MT>
+__device__ __forceinline__ void load_n8(uint32_t (&w)[MT][2][2], const uint8_t* rs_ptr,
+                                        const uint8_t* xs_ptr, uint32_t pitch, int g, int colc) {
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const uint32_t off = (mt * 16 + g + 8 * hh) * pitch + colc * 2;
+      w[mt][hh][0] = *reinterpret_cast<const uint32_t*>(rs_ptr + off);
+      w[mt][hh][1] = *reinterpret_cast<const uint32_t*>(xs_ptr + off);
+    }
+}
+
 // Epilogue of one n8 column block of the re-projection for the rows of one
-// m16 tile: h = (res + x) + corr, bf16 round in place (into the x slot),
-// row amax, optional fp32 store.
+// m16 tile: h = (res + x) + corr from the preloaded words, bf16 round in place
+// (into the x slot), row amax, optional fp32 store.
 template <bool F32OUT>
-__device__ __forceinline__ void finish_n8(const float (&acc)[4], const uint8_t* rs_ptr, uint8_t* xs_ptr,
+__device__ __forceinline__ void finish_n8(const float (&acc)[4], const uint32_t (&w)[2][2], uint8_t* xs_ptr,
                                           uint32_t pitch, int rowA, int colc, float (&rmax)[2],
                                           void* h_out, int row0, int N, int D, int col0) {
 #pragma unroll
   for (int hh = 0; hh < 2; ++hh) {
     const int row = rowA + 8 * hh;
     const uint32_t off = row * pitch + colc * 2;
-    const uint32_t rw = *reinterpret_cast<const uint32_t*>(rs_ptr + off);
-    const uint32_t xw = *reinterpret_cast<const uint32_t*>(xs_ptr + off);
+    const uint32_t rw = w[hh][0], xw = w[hh][1];
     const float h0 = (bf16_lo_f32(rw) + bf16_lo_f32(xw)) + acc[2 * hh];
     const float h1 = (bf16_hi_f32(rw) + bf16_hi_f32(xw)) + acc[2 * hh + 1];
     const uint32_t hb = pack_bf16x2(h0, h1);
@@ -720,6 +735,8 @@ boundary_cluster_smem_kernel(const bf16* __restrict__ x, const bf16* __restrict_
       for (int mt = 0; mt < C::MT; ++mt) rmax[mt][0] = rmax[mt][1] = 0.f;
 
       const int ntw = Dc / 64;  // n8 tiles per warp
+      uint32_t wcur[C::MT][2][2];
+      load_n8<C::MT>(wcur, rs_ptr, xs_ptr, pitch, g, warp * ntw * 8 + 2 * q4);
       for (int t8 = 0; t8 < ntw; ++t8) {
         const int d0 = (warp * ntw + t8) * 8;
         uint32_t b[C::KS2][2];
@@ -744,17 +761,30 @@ boundary_cluster_smem_kernel(const bf16* __restrict__ x, const bf16* __restrict_
                           b[2 * p + 1][0], b[2 * p + 1][1]);
           }
         }
+        float acc[C::MT][4];
 #pragma unroll
         for (int mt = 0; mt < C::MT; ++mt) {
-          float acc[4] = {0.f, 0.f, 0.f, 0.f};
+          acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
 #pragma unroll
           for (int ks = 0; ks < C::KS2; ++ks) {
-            mma_bf16_16816(acc, ahi[mt][ks], b[ks][0], b[ks][1]);
-            mma_bf16_16816(acc, alo[mt][ks], b[ks][0], b[ks][1]);
+            mma_bf16_16816(acc[mt], ahi[mt][ks], b[ks][0], b[ks][1]);
+            mma_bf16_16816(acc[mt], alo[mt][ks], b[ks][0], b[ks][1]);
           }
-          finish_n8<F32OUT>(acc, rs_ptr, xs_ptr, pitch, mt * 16 + g, d0 + 2 * q4, rmax[mt], h_out, row0,
-                            N, D, col0);
         }
+        // next block's words (the last block re-reads its own) before this block's stores
+        uint32_t wnext[C::MT][2][2];
+        load_n8<C::MT>(wnext, rs_ptr, xs_ptr, pitch, g, (t8 + 1 < ntw ? d0 + 8 : d0) + 2 * q4);
+#pragma unroll
+        for (int mt = 0; mt < C::MT; ++mt)
+          finish_n8<F32OUT>(acc[mt], wcur[mt], xs_ptr, pitch, mt * 16 + g, d0 + 2 * q4, rmax[mt], h_out, row0,
+                            N, D, col0);
+#pragma unroll
+        for (int mt = 0; mt < C::MT; ++mt)
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            wcur[mt][hh][0] = wnext[mt][hh][0];
+            wcur[mt][hh][1] = wnext[mt][hh][1];
+          }
       }
       publish_amax<C::MT, T>(rmax, wamax, amaxbuf, warp, lane, tid);
     }
