@@ -21,6 +21,7 @@
 #include "boundary_kernels.cuh"
 #include "boundary_rowtile.cuh"
 #include "w4a4_gemm_kernels.cuh"
+#include "w4a4_gemm_skinny.cuh"
 
 using namespace respin;
 
@@ -313,6 +314,41 @@ respin_status_t check_device(int want) {
 
 }  // namespace
 
+// Up to 128 tokens the weight stream is the bound and w4a4_gemm_skinny_kernel
+// spreads it over O / 16 CTAs. Measured on B200 (K = O = 4096, CUDA-graph
+// replay, weights larger than L2), skinny vs the tensor-memory kernel:
+// N = 1: 4.1 vs 11.6 us, 64: 8.6 vs 16.9 us, 128: 14.3 vs 21.4 us; from 160
+// tokens on the CTA-pair tiles win (19.4 us, flat up to 512 tokens; a
+// 256-token skinny variant took 22-27 us and single CTAs with K split over a
+// cluster 22-24 us there).
+#ifndef RESPIN_GEMM_SKINNY_MAX_TOKENS
+#define RESPIN_GEMM_SKINNY_MAX_TOKENS 128
+#endif
+static_assert(RESPIN_GEMM_SKINNY_MAX_TOKENS <= 128, "the skinny GEMM holds at most 128 tokens per CTA");
+
+template <int NT, int TG>
+static cudaError_t launch_skinny(const uint8_t* qa, const float* sa, const uint8_t* qw, const float* sw, int N,
+                                 int K, int O, void* out, cudaStream_t s, bool i32) {
+  const dim3 grid(static_cast<unsigned>(O / kSkRows)), block(kSkThreads);
+  if (i32)
+    w4a4_gemm_skinny_kernel<NT, TG, true><<<grid, block, 0, s>>>(qa, sa, qw, sw, N, K, O, out);
+  else
+    w4a4_gemm_skinny_kernel<NT, TG, false><<<grid, block, 0, s>>>(qa, sa, qw, sw, N, K, O, out);
+  return cudaGetLastError();
+}
+
+static respin_status_t gemm_skinny(const uint8_t* qa, const float* sa, const uint8_t* qw, const float* sw, int N,
+                                   int K, int O, void* out, cudaStream_t s, bool i32) {
+  cudaError_t e;
+  if (N <= 8) e = launch_skinny<1, 1>(qa, sa, qw, sw, N, K, O, out, s, i32);
+  else if (N <= 16) e = launch_skinny<2, 1>(qa, sa, qw, sw, N, K, O, out, s, i32);
+  else if (N <= 32) e = launch_skinny<4, 1>(qa, sa, qw, sw, N, K, O, out, s, i32);
+  else if (N <= 64) e = launch_skinny<4, 2>(qa, sa, qw, sw, N, K, O, out, s, i32);
+  else e = launch_skinny<4, 4>(qa, sa, qw, sw, N, K, O, out, s, i32);
+  if (e != cudaSuccess) return cuda_fail(e, "w4a4_gemm_skinny_kernel launch");
+  return ok();
+}
+
 extern "C" {
 
 const char* respin_last_error(void) { return t_last_error.c_str(); }
@@ -512,20 +548,10 @@ respin_status_t respin_boundary_forward(respin_plan_t plan, const void* x, const
 }
 
 extern "C++" {
-template <int CG, bool I32, int SPLIT = 1>
+template <int CG, bool I32>
 const void* gemm_fn() {
-  return reinterpret_cast<const void*>(&w4a4_gemm_kernel<CG, I32, SPLIT>);
+  return reinterpret_cast<const void*>(&w4a4_gemm_kernel<CG, I32>);
 }
-}
-
-// Split-K kernels (single CTAs): SPLIT in {2, 4, 8}.
-static const void* gemm_split_fn(int split, bool i32) {
-  switch (split) {
-    case 2: return i32 ? gemm_fn<1, true, 2>() : gemm_fn<1, false, 2>();
-    case 4: return i32 ? gemm_fn<1, true, 4>() : gemm_fn<1, false, 4>();
-    case 8: return i32 ? gemm_fn<1, true, 8>() : gemm_fn<1, false, 8>();
-    default: return nullptr;
-  }
 }
 
 // The GEMM kernels need the large dynamic shared-memory carve-out; set it
@@ -534,7 +560,6 @@ struct GemmDeviceInfo {
   bool ready = false;
   int sms = 0;
   int max_pairs = 0;
-  int max_split4 = 0;   // co-resident clusters of 4 single CTAs
 };
 
 static cudaError_t gemm_prepare(int dev, GemmDeviceInfo* info) {
@@ -545,13 +570,9 @@ static cudaError_t gemm_prepare(int dev, GemmDeviceInfo* info) {
   GemmDeviceInfo& d = infos[dev];
   if (!d.ready) {
     cudaError_t e = cudaSuccess;
-    const void* fns[10] = {gemm_fn<1, false>(), gemm_fn<1, true>(), gemm_fn<2, false>(), gemm_fn<2, true>(),
-                           gemm_split_fn(2, false), gemm_split_fn(2, true), gemm_split_fn(4, false),
-                           gemm_split_fn(4, true), gemm_split_fn(8, false), gemm_split_fn(8, true)};
-    const int smem[10] = {GemmCfg<1>::Smem, GemmCfg<1>::Smem, GemmCfg<2>::Smem, GemmCfg<2>::Smem,
-                          GemmCfg<1>::Smem, GemmCfg<1>::Smem, GemmCfg<1>::Smem,
-                          GemmCfg<1>::Smem, GemmCfg<1>::Smem, GemmCfg<1>::Smem};
-    for (int i = 0; i < 10 && e == cudaSuccess; ++i)
+    const void* fns[4] = {gemm_fn<1, false>(), gemm_fn<1, true>(), gemm_fn<2, false>(), gemm_fn<2, true>()};
+    const int smem[4] = {GemmCfg<1>::Smem, GemmCfg<1>::Smem, GemmCfg<2>::Smem, GemmCfg<2>::Smem};
+    for (int i = 0; i < 4 && e == cudaSuccess; ++i)
       e = cudaFuncSetAttribute(fns[i], cudaFuncAttributeMaxDynamicSharedMemorySize, smem[i]);
     if (e != cudaSuccess) return e;
     e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
@@ -570,13 +591,6 @@ static cudaError_t gemm_prepare(int dev, GemmDeviceInfo* info) {
     if (cudaOccupancyMaxActiveClusters(&d.max_pairs, fns[2], &lc) != cudaSuccess) {
       cudaGetLastError();
       d.max_pairs = 0;
-    }
-    attr[0].val.clusterDim.x = 4;
-    lc.gridDim = dim3(4, 1, 1);
-    lc.dynamicSmemBytes = GemmCfg<1>::Smem;
-    if (cudaOccupancyMaxActiveClusters(&d.max_split4, fns[6], &lc) != cudaSuccess) {
-      cudaGetLastError();
-      d.max_split4 = 0;
     }
     d.ready = true;
   }
@@ -631,13 +645,15 @@ static respin_status_t gemm_common(const uint8_t* q_act, const float* scale_act,
     return fail(RESPIN_ERR_ALIGNMENT, "scale_act must be 4-byte and scale_w 16-byte aligned");
   if (fault_at("launch")) return fail(RESPIN_ERR_CUDA, "injected fault at launch");
 
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (N <= RESPIN_GEMM_SKINNY_MAX_TOKENS) return gemm_skinny(q_act, scale_act, q_w, scale_w, N, K, O, out, s, i32);
+
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
   GemmDeviceInfo info;
   e = gemm_prepare(dev, &info);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gemm smem)");
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
   // CTA pairs (256-token tiles) from this many tokens on.
 #ifndef RESPIN_GEMM_PAIR_MIN_TOKENS
 #define RESPIN_GEMM_PAIR_MIN_TOKENS (kGemmBM + 1)
@@ -650,31 +666,17 @@ static respin_status_t gemm_common(const uint8_t* q_act, const float* scale_act,
       !make_tmap_u8(&tmB, q_w, O, K / 2, kGemmBN / CG, kGemmBK / 2) ||
       !make_tmap_out(&tmO, out, N, O, i32))
     return fail(RESPIN_ERR_CUDA, "cuTensorMapEncodeTiled failed for the GEMM operands or output");
-  // Split K for few single-CTA tiles (small N): a cluster of SPLIT CTAs per
-  // tile, one tile per cluster, so that the K loop is spread over more SMs.
-  // Every CTA sends its whole 128 x 256 partial through distributed shared
-  // memory, so the split pays off only up to 4 and only while all clusters
-  // are co-resident (measured on B200: 4096 x 4096, 8 tokens: 26.1 us
-  // unsplit, 21.1 us split 2, 19.6 us split 4, 43 us split 8).
-  int split = 1;
-  if (CG == 1) {
-    const int KBt = K / kGemmBK;
-    if (KBt % 4 == 0 && KBt >= 16 && 4 * tiles <= 4 * info.max_split4) split = 4;
-    else if (KBt % 2 == 0 && KBt >= 8 && 2 * tiles <= info.sms) split = 2;
-  }
-  const void* fn = split > 1 ? gemm_split_fn(split, i32)
-                   : CG == 2 ? (i32 ? gemm_fn<2, true>() : gemm_fn<2, false>())
-                             : (i32 ? gemm_fn<1, true>() : gemm_fn<1, false>());
-  const long long groups = split > 1 ? tiles
-                           : CG == 2 ? (tiles < info.max_pairs ? tiles : info.max_pairs)
-                                     : (tiles < info.sms ? tiles : info.sms);
+  const void* fn = CG == 2 ? (i32 ? gemm_fn<2, true>() : gemm_fn<2, false>())
+                           : (i32 ? gemm_fn<1, true>() : gemm_fn<1, false>());
+  const long long groups = CG == 2 ? (tiles < info.max_pairs ? tiles : info.max_pairs)
+                                   : (tiles < info.sms ? tiles : info.sms);
   cudaLaunchConfig_t lc = {};
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = CG * split;
+  attr[0].val.clusterDim.x = CG;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
-  lc.gridDim = dim3(static_cast<unsigned>(groups * CG * split), 1, 1);
+  lc.gridDim = dim3(static_cast<unsigned>(groups * CG), 1, 1);
   lc.blockDim = dim3(kGemmThreads, 1, 1);
   lc.dynamicSmemBytes = CG == 2 ? GemmCfg<2>::Smem : GemmCfg<1>::Smem;
   lc.stream = s;

@@ -45,13 +45,6 @@
 //    every SM widens and stores half the weight bytes it would alone;
 //  * 4 epilogue warps drain the other TMEM buffer (tcgen05.ld), apply the two
 //    scales and store bf16, overlapping the next tile's main loop.
-// Split K (SPLIT > 1, single CTAs, few tiles - e.g. decode): a cluster of
-// SPLIT CTAs computes one tile, CTA k over K blocks [k KB/S, (k+1) KB/S).
-// After a cluster barrier (every CTA's MMAs are done, so the widened and
-// packed stage rings, contiguous from the base, are free) each CTA writes its
-// partial int32 accumulators of the columns that CTA j owns (256/S of them)
-// into CTA j's rings with distributed-shared-memory stores; after a second barrier CTA j sums the S partials in rank order
-// (exact, deterministic) and runs the usual epilogue on its columns.
 #pragma once
 
 #include <cuda.h>
@@ -130,15 +123,12 @@ __device__ __forceinline__ uint32_t sw64_offset(int r, int j) {
 // (inner dimension first), no swizzle, out-of-range elements zero filled.
 // tmO: the output [N, O] (bf16, or int32 for I32OUT), box {64 bytes, 32 rows},
 // 64-byte swizzle; the store clips rows >= N and columns >= O.
-template <int CG, bool I32OUT, int SPLIT = 1>
+template <int CG, bool I32OUT>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const __grid_constant__ CUtensorMap tmO, const float* __restrict__ sa,
                  const float* __restrict__ sw, int N, int K, int O) {
   using G = GemmCfg<CG>;
-  static_assert(SPLIT == 1 || CG == 1, "split K runs on single CTAs");
-  static_assert(SPLIT == 1 || SPLIT * (kGemmBM * kGemmBN * 4 / SPLIT) <= G::US * G::Stage + G::PS * G::PStage,
-                "split-K receive slots fit in the (idle) stage rings");
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -157,13 +147,9 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t rank = CG == 2 ? cluster_ctarank() : 0u;
-  constexpr int CL = CG * SPLIT;   // CTAs per cluster
-  const int group = static_cast<int>(blockIdx.x) / CL;
-  const int ngroups = static_cast<int>(gridDim.x) / CL;
-  // K blocks of this CTA: all of them, or its share of a split-K cluster
-  const uint32_t krank = SPLIT > 1 ? cluster_ctarank() : 0u;
-  const int KB = K / kGemmBK / SPLIT;
-  const int kb0 = static_cast<int>(krank) * KB;
+  const int group = static_cast<int>(blockIdx.x) / CG;
+  const int ngroups = static_cast<int>(gridDim.x) / CG;
+  const int KB = K / kGemmBK;   // K blocks
   const int mtiles = (N + G::TileM - 1) / G::TileM;
   const int ntiles = (O + kGemmBN - 1) / kGemmBN;
   const int tiles = mtiles * ntiles;
@@ -335,8 +321,8 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
           if (!ok) continue;
           const uint32_t dst = pbase + ps * G::PStage;
           mbar_arrive_expect_tx(pfull0 + 8 * ps, bytes);
-          if (is_b) tma_load_2d(dst + G::PAStage, &tmB, (kb0 + kb) * (kGemmBK / 2), brow, pfull0 + 8 * ps);
-          else tma_load_2d(dst, &tmA, (kb0 + kb) * (kGemmBK / 2), arow, pfull0 + 8 * ps);
+          if (is_b) tma_load_2d(dst + G::PAStage, &tmB, kb * (kGemmBK / 2), brow, pfull0 + 8 * ps);
+          else tma_load_2d(dst, &tmA, kb * (kGemmBK / 2), arow, pfull0 + 8 * ps);
         }
       }
     }
@@ -389,7 +375,7 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     float* sws = reinterpret_cast<float*>(smem + (swbase - base) + quad * G::SwBytes);
     bool ok = true;
     int local = 0;
-    for (int t = group; SPLIT == 1 && t < tiles; t += ngroups, ++local) {
+    for (int t = group; t < tiles; t += ngroups, ++local) {
       const int ab = local & 1;
       const int m0 = (t / ntiles) * G::TileM + static_cast<int>(rank) * kGemmBM;
       const int n0 = (t % ntiles) * kGemmBN;
@@ -437,70 +423,9 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         else mbar_arrive(aempty0 + 8 * ab);
       }
     }
-    if constexpr (SPLIT > 1) {
-      // one tile per cluster: its accumulators, then the reduction below
-      if (group < tiles && ok) ok = mbar_wait(afull0, 0, kSiteGemmAccum);
-    }
     // the staging units must not be released while a store still reads them
     if (lane == 0) bulk_wait_group_all();
     __syncwarp();
-  }
-  if constexpr (SPLIT > 1) {
-    // ---------------------------------------------- split-K reduction
-    constexpr int OC = kGemmBN / SPLIT;          // columns each CTA finishes
-    constexpr int SLOT = kGemmBM * OC * 4;       // one partial: 128 rows x OC int32
-    const bool live = group < tiles;
-    const int m0 = (group / ntiles) * G::TileM, n0 = (group % ntiles) * kGemmBN;
-    const int row = quad * 32 + lane;
-    // 16-byte piece pi of a row slot stored at (pi & ~7) | ((pi ^ row) & 7):
-    // the 32 lanes of a warp (32 rows) spread over 8 bank groups
-    auto pos16 = [&](int pi) { return ((pi & ~7) | ((pi ^ row) & 7)) * 16; };
-    tc_fence_before();
-    cluster_sync();   // every CTA's MMAs are done: its stage ring may be overwritten
-    if (warp >= kGemmEpiWarp0 && live) {
-      tc_fence_after();
-      const uint32_t tb = tmem + (static_cast<uint32_t>(quad * 32) << 16);
-#pragma unroll 1
-      for (int cc = 0; cc < kGemmBN / 32; ++cc) {
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(tb + cc * 32, v);
-        tmem_wait_ld();
-        const uint32_t owner = static_cast<uint32_t>(cc * 32 / OC);
-        const int p0 = (cc * 32 % OC) / 4;       // first 16-byte piece in the owner's row slot
-        if (m0 + row >= N) continue;   // rows past N are never stored: not sent either
-        const uint32_t dst = map_to_rank(base + krank * SLOT + row * (OC * 4), owner);
-#pragma unroll
-        for (int p = 0; p < 8; ++p)
-          st_dsmem_u32x4(dst + pos16(p0 + p), make_uint4(v[4 * p], v[4 * p + 1], v[4 * p + 2], v[4 * p + 3]));
-      }
-    }
-    cluster_sync();   // all partials delivered
-    if (warp >= kGemmEpiWarp0 && live) {
-      const int y = m0 + quad * 32;
-      const float sa_r = (!I32OUT && m0 + row < N) ? __ldg(sa + m0 + row) : 0.f;
-#pragma unroll 1
-      for (int cg = 0; cg < OC / 32; ++cg) {
-        uint32_t v[32];
-#pragma unroll
-        for (int e = 0; e < 32; ++e) v[e] = 0u;
-        for (int sl = 0; m0 + row < N && sl < SPLIT; ++sl) {   // rank order: the same sum on every call
-          const uint8_t* src = smem + sl * SLOT + row * (OC * 4);
-#pragma unroll
-          for (int p = 0; p < 8; ++p) {
-            const uint4 w = *reinterpret_cast<const uint4*>(src + pos16(cg * 8 + p));
-            v[4 * p] += w.x;
-            v[4 * p + 1] += w.y;
-            v[4 * p + 2] += w.z;
-            v[4 * p + 3] += w.w;
-          }
-        }
-        const int colb = n0 + static_cast<int>(krank) * OC + cg * 32;
-        if (colb >= O || y >= N) continue;
-        store_chunk(v, colb, y, sa_r, I32OUT ? nullptr : sw + colb);   // channel scales read from global
-      }
-      if (lane == 0) bulk_wait_group_all();
-      __syncwarp();
-    }
   }
   tc_fence_before();
   // Neither CTA of a pair may release its TMEM or shared memory while the

@@ -1,4 +1,5 @@
-"""GPU parity of the tcgen05 W4A4 GEMM against the exact-integer oracle.
+"""GPU parity of the W4A4 GEMM kernels (skinny kernel for N <= 128 tokens,
+tensor-memory kernel above) against the exact-integer oracle.
 
 W4A4 linear (ReSpinQuant explainers zh §3-§4, fr §4): int32 accumulators
 must be bit-exact; the bf16 output of the binary32 scale epilogue must be
@@ -52,22 +53,55 @@ def check(qa, qw, sa, sw, acc, outb, rows=None):
 
 
 @pytest.mark.parametrize("N,K,O_", [
-    (1, 128, 16),          # smallest
-    (5, 256, 48),          # ragged everything
-    (128, 512, 256),       # exactly one tile
+    # tensor-memory kernel (more than 128 tokens; CTA pairs of 256 rows)
+    (129, 128, 16),        # smallest K and O
+    (133, 256, 48),        # ragged everything
+    (256, 512, 256),       # exactly one pair tile
     (200, 1024, 272),      # ragged M and N tiles, several K blocks
     (300, 4096, 512),
-    (64, 14336, 4096),     # down-projection K (stack workload)
-    # split K over clusters of single CTAs (few tiles)
-    (16, 1024, 4096),      # split 2 (8 K blocks)
-    (33, 4096, 4112),      # split 4; last tile 16 channels wide, ragged rows
-    (128, 2048, 272),      # split 4; owners of columns past O idle, full A tile
-    (3, 8192, 1040),       # split 4, 64 K blocks, 5 tiles
+    (129, 1024, 4096),     # one row past a single-CTA tile
+    (200, 4096, 4112),     # last tile 16 channels wide, ragged rows
+    (256, 2048, 272),      # exactly one pair tile of rows, ragged channels
+    (300, 8192, 1040),     # 64 K blocks, two row tiles
 ])
 def test_gemm_small(N, K, O_):
     qa, qw, sa, sw = make(N, K, O_)
     acc, outb = run(qa, qw, sa, sw)
     check(qa, qw, sa, sw, acc, outb)
+
+
+@pytest.mark.parametrize("N,K,O_", [
+    # skinny kernel (N <= 128): token tiles of 8 / 16 / 32 / 2 x 32 / 4 x 32
+    (1, 128, 16),          # one chunk: 7 of 8 warps hold no K
+    (7, 256, 32),
+    (9, 1152, 48),         # 9 chunks over 8 warps
+    (16, 4096, 11008),
+    (17, 4096, 4096),
+    (31, 14336, 4096),     # 112 chunks: 14 per warp, ragged last group
+    (33, 2048, 16),
+    (63, 4096, 272),
+    (64, 14336, 4096),     # down-projection K (stack workload)
+    (65, 8192, 1040),
+    (100, 1024, 4096),
+    (128, 2048, 272),
+])
+def test_gemm_skinny(N, K, O_):
+    qa, qw, sa, sw = make(N, K, O_, seed=3)
+    acc, outb = run(qa, qw, sa, sw)
+    check(qa, qw, sa, sw, acc, outb)
+
+
+def test_gemm_skinny_extremes_exact():
+    """Skinny kernel at the largest K: all codes -8 gives acc = 64 K = 2^22
+    (the MMA sums 2^30 before the shift back)."""
+    N, K, O_ = 9, 65536, 16
+    qa = np.full((N, K // 2), 0x88, np.uint8)
+    qw = np.full((O_, K // 2), 0x88, np.uint8)
+    acc, _ = run(qa, qw, np.ones(N, np.float32), np.ones(O_, np.float32))
+    assert np.all(acc == 64 * K)
+    qw2 = np.full((O_, K // 2), 0x77, np.uint8)
+    acc2, _ = run(qa, qw2, np.ones(N, np.float32), np.ones(O_, np.float32))
+    assert np.all(acc2 == -56 * K)
 
 
 @pytest.mark.parametrize("N", [1, 8, 32, 64, 256])
@@ -95,7 +129,8 @@ def test_gemm_full_size_llama3_8b_down_sampled():
 
 
 def test_gemm_extremes_exact():
-    """All codes -8 (largest magnitude): acc = 64 K exactly."""
+    """All codes -8 (largest magnitude): acc = 64 K exactly (tensor-memory
+    kernel)."""
     N, K, O_ = 130, 14336, 32
     qa = np.full((N, K // 2), 0x88, np.uint8)
     qw = np.full((O_, K // 2), 0x88, np.uint8)
@@ -108,9 +143,11 @@ def test_gemm_extremes_exact():
     assert np.all(acc2 == -56 * K)
 
 
-def test_gemm_selection_matrix():
-    """One +1 per weight row: the GEMM gathers activation codes."""
-    N, K, O_ = 70, 512, 64
+@pytest.mark.parametrize("N", [20, 70])
+def test_gemm_selection_matrix(N):
+    """One +1 per weight row: the GEMM gathers activation codes (skinny and
+    tensor-memory kernels)."""
+    K, O_ = 512, 64
     rs = np.random.default_rng(9)
     qa = W.int4_packed_random(N, K, 4, W.TID_ACODES)
     sel = rs.integers(0, K, O_)
