@@ -135,7 +135,9 @@ respin_status_t respin_boundary_forward(respin_plan_t plan, const void* x,
  *   O         : output channels; O % 16 == 0, O >= 16.
  *   out       : bf16 [N, O] (device).
  * Both products of the epilogue round to nearest even in binary32; the
- * integer sum is exact. Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, CUDA.
+ * integer sum is exact, so the result does not depend on which kernel runs
+ * (N <= 128: weight-streaming kernel; above: tensor-memory tiles).
+ * Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, CUDA.
  */
 respin_status_t w4a4_gemm(const uint8_t* q_act, const float* scale_act,
                           const uint8_t* q_w, const float* scale_w, int N,
