@@ -30,6 +30,12 @@ What the pages fix, and how this module follows it:
   all in IEEE binary32, on the bfloat16-rounded boundary output ``g``. Tokens
   with ``amax < 2^-125`` get scale 0 and all-zero codes (below that
   ``7 / amax`` would overflow binary32).
+* 3-bit activations (W3A3, named beside W4A4 in zh §3-§4, it §3, nl §3 and
+  fr §4; no quantizer given either). Reading: the same per-token symmetric
+  form with bound 3 instead of 7: ``inv = 3 / amax``,
+  ``q = clamp(rint(g * inv), -4, 3)``, ``scale = amax / 3``; codes stay in
+  4-bit containers (the pages give no 3-bit packing), so the integer GEMM is
+  the same for both widths.
 * Packing: element ``2j`` in the low nibble of byte ``j``, element ``2j+1`` in
   the high nibble, two's complement.
 * W4A4 GEMM: ``acc[n, o] = sum_k a[n, k] w[o, k]`` exactly in integers, then
@@ -191,31 +197,45 @@ def bf16_bits_to_f32(bits) -> np.ndarray:
 
 
 # --------------------------------------------------------------------------
-# Per-token symmetric INT4 quantizer (binary32)
+# Per-token symmetric INT4 / INT3 quantizer (binary32)
 # --------------------------------------------------------------------------
 
-def quantize_int4_per_token(g) -> tuple[np.ndarray, np.ndarray]:
-    """(codes int8 [N, D], scale float32 [N]) for float32 [N, D] input ``g``.
+def quantize_per_token(g, qmax: int) -> tuple[np.ndarray, np.ndarray]:
+    """(codes int8 [N, D], scale float32 [N]) for float32 [N, D] input ``g``
+    with ``qmax`` = 7 (INT4) or 3 (INT3).
 
     Every operation is one IEEE binary32 operation with round to nearest even:
-    amax = max |g|; inv = 7 / amax; q = clamp(rint(g * inv), -8, 7);
-    scale = amax / 7. A token with amax < 2^-125 gets scale 0 and zero codes.
+    amax = max |g|; inv = qmax / amax; q = clamp(rint(g * inv), -qmax-1, qmax);
+    scale = amax / qmax. A token with amax < 2^-125 gets scale 0 and zero
+    codes.
     """
+    if qmax not in (7, 3):
+        raise ValueError("qmax must be 7 (INT4) or 3 (INT3)")
     g = np.asarray(g, np.float32)
     N, D = g.shape
     codes = np.zeros((N, D), np.int8)
     scale = np.zeros(N, np.float32)
-    seven = np.float32(7.0)
+    qm = np.float32(qmax)
     for n in range(N):
         amax = np.float32(np.max(np.abs(g[n]))) if D else np.float32(0)
         if not amax >= ZERO_TOKEN_AMAX:
             continue
-        inv = np.float32(seven / amax)
+        inv = np.float32(qm / amax)
         t = (g[n] * inv).astype(np.float32)
         q = np.rint(t)
-        codes[n] = np.clip(q, -8, 7).astype(np.int8)
-        scale[n] = np.float32(amax / seven)
+        codes[n] = np.clip(q, -qmax - 1, qmax).astype(np.int8)
+        scale[n] = np.float32(amax / qm)
     return codes, scale
+
+
+def quantize_int4_per_token(g) -> tuple[np.ndarray, np.ndarray]:
+    """W4A4 activations: quantize_per_token with bound 7."""
+    return quantize_per_token(g, 7)
+
+
+def quantize_int3_per_token(g) -> tuple[np.ndarray, np.ndarray]:
+    """W3A3 activations: quantize_per_token with bound 3."""
+    return quantize_per_token(g, 3)
 
 
 def pack_int4(codes) -> np.ndarray:
@@ -291,17 +311,18 @@ def plan_factors(U, V):
             round_to_bf16(np.asarray(V, np.float32)))
 
 
-def boundary_reference(x, residual, U32, V32):
+def boundary_reference(x, residual, U32, V32, qmax: int = 7):
     """Full reference for one boundary call with float32 host factors.
 
     Returns (h64, h_bf16_bits, codes, scale): h64 is the float64 fix with the
     plan's bfloat16 factors, h_bf16_bits its bfloat16 rounding, and the codes /
-    scales come from the quantizer applied to that bfloat16 output.
+    scales come from the quantizer (bound qmax) applied to that bfloat16
+    output.
     """
     Uq, Vq = plan_factors(U32, V32)
     h64 = boundary_fp64(x, residual, Uq, Vq)
     hb = bf16_bits(h64)
-    codes, scale = quantize_int4_per_token(bf16_bits_to_f32(hb))
+    codes, scale = quantize_per_token(bf16_bits_to_f32(hb), qmax)
     return h64, hb, codes, scale
 
 

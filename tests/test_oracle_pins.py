@@ -238,32 +238,54 @@ def test_quantizer_golden_cases():
     for p in gold["packing"]:
         assert O.pack_int4(np.array(p["codes"])).tolist() == p["bytes"]
         assert O.unpack_int4(np.array(p["bytes"], np.uint8)).tolist() == p["codes"]
+    for t in gold["int3_tokens"]:
+        codes, scale = O.quantize_int3_per_token(np.array([t["g"]], np.float32))
+        assert codes[0].tolist() == t["codes"]
+        assert scale[0] == np.float32(t["scale"])
 
 
-def test_quantizer_invariants():
+@pytest.mark.parametrize("qmax", [7, 3])
+def test_quantizer_invariants(qmax):
     rs = np.random.default_rng(11)
     g = rs.standard_normal((64, 256)).astype(np.float32)
     g[:, 3] *= 50
     g[5] = 0.0
-    codes, scale = O.quantize_int4_per_token(g)
-    assert codes.min() >= -8 and codes.max() <= 7
+    codes, scale = O.quantize_per_token(g, qmax)
+    assert codes.min() >= -qmax - 1 and codes.max() <= qmax
     nz = np.any(g != 0, axis=1)
-    assert np.all(np.max(np.abs(codes[nz]), axis=1) == 7)
+    assert np.all(np.max(np.abs(codes[nz]), axis=1) == qmax)
     assert scale[5] == 0 and not np.any(codes[5])
     # dequantization error within half a step (plus binary32 slack), in fp64
     err = np.abs(g.astype(np.float64) - codes * scale[:, None].astype(np.float64))
     assert np.all(err <= scale[:, None] * (0.5 + 2e-6))
-    # and the code is the nearest integer to g * 7 / amax up to that slack
+    # and the code is the nearest integer to g * qmax / amax up to that slack
     amax = np.max(np.abs(g), axis=1).astype(np.float64)
-    t = g[nz] * (7.0 / amax[nz, None])
+    t = g[nz] * (qmax / amax[nz, None])
     assert np.all(np.abs(t - codes[nz]) <= 0.5 + 1e-5)
 
 
-def test_quantizer_tiny_amax_is_zero_token():
+def test_quantizer_int3_brute_force_nearest():
+    """INT3 codes are the nearest of the 8 levels -4..3 to g*3/amax, brute
+    force over the levels (ties, which have measure zero here, excluded)."""
+    rs = np.random.default_rng(21)
+    g = rs.standard_normal((32, 96)).astype(np.float32)
+    codes, scale = O.quantize_int3_per_token(g)
+    t = g.astype(np.float64) * (3.0 / np.max(np.abs(g), axis=1, keepdims=True))
+    levels = np.arange(-4, 4)
+    dist = np.abs(t[..., None] - levels)
+    best = levels[np.argmin(dist, axis=-1)]
+    srt = np.sort(dist, axis=-1)
+    clear = srt[..., 1] - srt[..., 0] > 1e-5
+    assert np.array_equal(codes[clear], best[clear])
+    assert np.allclose(scale, np.max(np.abs(g), axis=1) / 3.0, rtol=2 ** -23)
+
+
+@pytest.mark.parametrize("qmax", [7, 3])
+def test_quantizer_tiny_amax_is_zero_token(qmax):
     g = np.array([[1e-38, -2e-38, 0.0, 0.0], [3e-38, 0, 0, 0]], np.float32)
-    codes, scale = O.quantize_int4_per_token(g)
+    codes, scale = O.quantize_per_token(g, qmax)
     assert scale[0] == 0 and not codes[0].any()
-    assert scale[1] > 0 and codes[1, 0] == 7
+    assert scale[1] > 0 and codes[1, 0] == qmax
 
 
 def test_pack_roundtrip():
