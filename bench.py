@@ -30,6 +30,13 @@ if ROOT not in sys.path:
 
 METRIC = "tokens/s fused ΔT-lowrank+INT4 quant (D=4096,r=32); W4A4 GEMM TOPS"
 WORKLOAD = "llama2_7b"
+# The headline step in its two quantization settings: activation (and weight)
+# code width per --workload name.
+STEP_BITS = {"llama2_7b": 4, "llama2_7b_w3a3": 3}
+
+
+def metric(bits: int) -> str:
+    return METRIC if bits == 4 else METRIC.replace("INT4", "INT3").replace("W4A4", "W3A3")
 NSETS = 4            # rotating input sets: 4 x 56 MB > 126 MB L2
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
@@ -49,10 +56,12 @@ def parse_args():
     p.add_argument("--tokens", type=int, default=None,
                    help="tokens for --profile-launch (default 2048)")
     p.add_argument("--workload", default="llama2_7b",
-                   choices=["llama2_7b", "tiny", "decode", "llama2_70b", "llama3_8b_stack"],
-                   help="llama2_7b (default): the headline step. The others print "
-                        "one JSON line each for the remaining workload configurations "
-                        "(1 GPU)")
+                   choices=["llama2_7b", "llama2_7b_w3a3", "tiny", "decode", "llama2_70b",
+                            "llama3_8b_stack"],
+                   help="llama2_7b (default): the headline step; llama2_7b_w3a3: the "
+                        "same step with 3-bit activation and weight codes. The others "
+                        "print one JSON line each for the remaining workload "
+                        "configurations (1 GPU)")
     return p.parse_args()
 
 
@@ -134,7 +143,7 @@ class ClockSampler(threading.Thread):
 
 # ---------------------------------------------------------------- oracle legs
 
-def oracle_sample_rate(fx, qw, sw, n_boundary: int, n_gemm: int):
+def oracle_sample_rate(fx, qw, sw, n_boundary: int, n_gemm: int, bits: int = 4):
     """Time the CPU oracle (as it stands) on a bounded sample; tokens/s of
     the whole path per token = 1 / (t_boundary/token + t_gemm/token)."""
     import numpy as np
@@ -146,7 +155,7 @@ def oracle_sample_rate(fx, qw, sw, n_boundary: int, n_gemm: int):
         res = fx.residual[:n_boundary].float().numpy()
         U32, V32 = fx.U.astype(np.float32), fx.V.astype(np.float32)
         t0 = time.perf_counter()
-        _, _, codes, scale = O.boundary_reference(x, res, U32, V32)
+        _, _, codes, scale = O.boundary_reference(x, res, U32, V32, 7 if bits == 4 else 3)
         t1 = time.perf_counter()
         qa = O.pack_int4(codes[:n_gemm])
         acc = O.w4a4_acc(qa, qw)
@@ -170,23 +179,27 @@ def host_cpu() -> str:
     return "%s, %d logical cores" % (model, os.cpu_count() or 0)
 
 
-def cpu_baseline_block(fx, qw, sw):
-    rate, secs = oracle_sample_rate(fx, qw, sw, 2048, 160)
+def cpu_baseline_block(fx, qw, sw, bits: int = 4):
+    rate, secs = oracle_sample_rate(fx, qw, sw, 2048, 160, bits)
     return {"value": rate, "unit": "tokens/s", "cores": 1, "kind": "oracle", "cpu": host_cpu(),
-            "sample": "boundary oracle (fp64 fix + binary32 quantizer) on all "
-                      "2048 tokens, W4A4 GEMM oracle (exact int64 + binary32 "
+            "sample": "boundary oracle (fp64 fix + binary32 INT%d quantizer) on all "
+                      "2048 tokens, W%dA%d GEMM oracle (exact int64 + binary32 "
                       "epilogue) on 160 of the 2048 rows x 11008 channels; "
                       "per-token times summed; %.1f s of CPU work, 1 thread"
-                      % secs}
+                      % (bits, bits, bits, secs)}
 
 
-def workload_inputs(device: str | None):
+def weight_codes(W, bits: int, rows: int, K: int, seed: int):
+    return (W.int4_packed_random if bits == 4 else W.int3_packed_random)(rows, K, seed, W.TID_WEIGHTS)
+
+
+def workload_inputs(device: str | None, bits: int = 4):
     import numpy as np
     import workloads as W
     w = W.WORKLOADS[WORKLOAD]
     fx = W.workload_fixture(WORKLOAD)
     K = w.D
-    qw = W.int4_packed_random(w.O, K, 0, W.TID_WEIGHTS)
+    qw = weight_codes(W, bits, w.O, K, 0)
     sw = W.weight_scales(w.O, K, 0)
     return w, fx, qw, sw
 
@@ -195,26 +208,27 @@ def run_reference(args, rank: int):
     """The reference arm: the CPU oracle, timed on the host cores."""
     if rank != 0:
         return
-    w, fx, qw, sw = workload_inputs(None)
+    bits = STEP_BITS.get(args.workload, 4)
+    w, fx, qw, sw = workload_inputs(None, bits)
     nb, ng = 64, 4
     for _ in range(max(0, args.warmup)):
-        oracle_sample_rate(fx, qw, sw, nb, ng)
+        oracle_sample_rate(fx, qw, sw, nb, ng, bits)
     t = 0.0
     rates = []
     for _ in range(args.steps):
-        r, s = oracle_sample_rate(fx, qw, sw, nb, ng)
+        r, s = oracle_sample_rate(fx, qw, sw, nb, ng, bits)
         rates.append(r)
         t += s
     # per step: the full 2048-token batch at the sampled per-token cost
     per_tok = sum(1.0 / r for r in rates) / len(rates)
     value = 1.0 / per_tok
     line = {
-        "impl": "reference", "metric": METRIC, "value": value,
+        "impl": "reference", "metric": metric(bits), "value": value,
         "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": per_tok * w.N * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64+f32+int64", "data": "synthetic",
-        "config": config_block(w, args.gpus),
+        "config": config_block(w, args.gpus, bits),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1,
                          "kind": "oracle", "cpu": host_cpu(),
                          "sample": "each step: boundary oracle on 64 tokens "
@@ -226,9 +240,10 @@ def run_reference(args, rank: int):
     print(json.dumps(line), flush=True)
 
 
-def config_block(w, n_gpus):
-    return {"workload": "Llama-2-7B-shaped boundary + W4A4 GEMM: D=4096, "
-                        "2048 tokens/GPU, r=32, GEMM 4096->11008",
+def config_block(w, n_gpus, bits: int = 4):
+    return {"workload": "Llama-2-7B-shaped boundary + W%dA%d GEMM: D=4096, "
+                        "2048 tokens/GPU, r=32, GEMM 4096->11008" % (bits, bits),
+            "act_bits": bits, "weight_bits": bits,
             "D": w.D, "tokens_per_gpu": w.N, "r": w.r, "gemm_out": w.O,
             "global_batch": w.N * n_gpus, "parallelism": "dp%d" % n_gpus,
             "l2": "inputs larger than L2: %d rotating input sets of %.0f MB"
@@ -308,10 +323,12 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     torch.cuda.set_device(dev)
     dist = init_dist("nccl", dev) if world > 1 else None
 
-    w, fx, qw_np, sw_np = workload_inputs("cuda")
+    bits = STEP_BITS[args.workload]
+    w, fx, qw_np, sw_np = workload_inputs("cuda", bits)
     D, N, r, O_ = w.D, w.N, w.r, w.O
     K = D
-    plan = rq.Plan(D, r, fx.U.astype(np.float32), fx.V.astype(np.float32))
+    plan = rq.Plan(D, r, fx.U.astype(np.float32), fx.V.astype(np.float32),
+                   rq.RESPIN_ACT_INT3 if bits == 3 else 0)
 
     sets = []
     for i in range(NSETS):
@@ -323,7 +340,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         if i == 0 and rank == 0:
             x.copy_(fx.x.to(dev))
             res.copy_(fx.residual.to(dev))
-        qw = torch.from_numpy(W.int4_packed_random(O_, K, i, W.TID_WEIGHTS)).to(dev)
+        qw = torch.from_numpy(weight_codes(W, bits, O_, K, i)).to(dev)
         sw = torch.from_numpy(W.weight_scales(O_, K, i)).to(dev)
         sets.append((x, res, qw, sw))
     h = torch.empty(N, D, dtype=torch.bfloat16, device=dev)
@@ -447,14 +464,14 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         b_bytes = N * (6.5 * D + 4) + 2 * D * 32 * 2
         b_gbs = b_bytes / (b_ms * 1e-3) / 1e9
         line = {
-            "metric": METRIC,
+            "metric": metric(bits),
             "value": job_tokens_per_s(world, N, ms_step),
             "unit": "tokens/s",
             "n_gpus": world, "steps": Ksteps, "warmup": args.warmup,
             "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "bf16+int4", "data": "synthetic",
-            "config": config_block(w, world),
+            "dtype": "bf16+int%d" % bits, "data": "synthetic",
+            "config": config_block(w, world, bits),
             "boundary_tokens_per_s": job_tokens_per_s(world, N, b_ms),
             "boundary_us": b_ms * 1e3,
             "gemm_tops": gemm_tops * world,
@@ -484,7 +501,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
             "clocks": clocks,
         }
         if world == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_baseline_block(fx, qw_np, sw_np)
+            line["cpu_baseline"] = cpu_baseline_block(fx, qw_np, sw_np, bits)
         print(json.dumps(line), flush=True)
     plan.destroy()
     if dist:
@@ -769,7 +786,7 @@ def main():
     if args.impl == "reference":
         run_reference(args, rank)
         return
-    if args.workload != "llama2_7b":
+    if args.workload not in STEP_BITS:
         run_workload(args)
         return
     run_ours(args, rank, world, local_rank)

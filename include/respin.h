@@ -57,6 +57,13 @@ typedef struct respin_plan_s* respin_plan_t;
  * bfloat16-rounded h'. Used to check the arithmetic of the fix directly. */
 #define RESPIN_H_FP32_DEBUG 1u
 
+/* Plan flag: 3-bit activation codes (W3A3, named beside W4A4 on the
+ * explainer pages: zh §3-§4, it §3, nl §3, fr §4; no quantizer is given
+ * there). The quantizer bound becomes 3 instead of 7: inv = 3 / amax,
+ * scale = amax / 3, codes in [-3, 3], stored in the same two's-complement
+ * nibbles, so w4a4_gemm consumes them (and 3-bit weight codes) unchanged. */
+#define RESPIN_ACT_INT3 2u
+
 /*
  * respin_plan_create -- prepare the rank-r fix of one block boundary.
  *
@@ -71,7 +78,7 @@ typedef struct respin_plan_s* respin_plan_t;
  *            residual + x followed by quantization.
  *   U_r    : HOST fp32 [D, r] row-major (may be NULL iff r == 0).
  *   V_r    : HOST fp32 [D, r] row-major (may be NULL iff r == 0).
- *   flags  : 0 or RESPIN_H_FP32_DEBUG.
+ *   flags  : 0, or RESPIN_H_FP32_DEBUG and/or RESPIN_ACT_INT3.
  *
  * The plan rounds U_r and V_r to bfloat16 (round to nearest even), copies
  * them to the current device (owned by the plan) and picks the launch
@@ -99,8 +106,9 @@ respin_status_t respin_plan_destroy(respin_plan_t plan);
  *     h[n]   = residual[n] + x[n] + y V_r^T
  *     h'[n]  = bf16(h[n])                            (round to nearest even)
  *     amax   = max_i |h'[n, i]|
- *     inv    = 7 / amax, scale[n] = amax / 7         (binary32, RN)
- *     q[n,i] = clamp(rint(h'[n,i] * inv), -8, 7)     (ties to even)
+ *     inv    = B / amax, scale[n] = amax / B         (binary32, RN)
+ *     q[n,i] = clamp(rint(h'[n,i] * inv), -B-1, B)   (ties to even)
+ * with B = 7 (INT4), or B = 3 for a plan made with RESPIN_ACT_INT3.
  * A token with amax < 2^-125 gets scale 0 and all-zero codes.
  *
  *   plan      : from respin_plan_create; its device must be current.

@@ -23,6 +23,7 @@ RESPIN_ERR_CUDA = 4
 RESPIN_ERR_OOM = 5
 RESPIN_ERR_DEVICE_CHECK = 6
 RESPIN_H_FP32_DEBUG = 1
+RESPIN_ACT_INT3 = 2
 
 # Every entry point include/respin.h declares (checked by the tests).
 EXPORTED = ("respin_plan_create", "respin_plan_destroy",

@@ -2,12 +2,13 @@
 //
 // Per token (row) n, with the plan's bfloat16 factors U (D x r) and V (D x r):
 //   y = residual[n] U ;  h = (residual[n] + x[n]) + y V^T  (fp32)
-//   h' = bf16(h) ; amax = max|h'| ; inv = 7/amax ; q = rint(h' inv)
+//   h' = bf16(h) ; amax = max|h'| ; inv = qmax/amax ; q = rint(h' inv)
 // This is the subspace residual rotation of the ReSpinQuant explainers (zh page
 // §2.2 steps 1-3: projection, transform inside the subspace, re-projection and
-// residual) in the row convention, followed by 4-bit activation quantization
-// (zh §3-§4, W4A4). Since |h'| <= amax, |fl(h' * fl(7/amax))| <= 7 (1+2^-24)^2
-// < 7.5, so the code is always in [-7, 7] and no clamp is needed.
+// residual) in the row convention, followed by 4-bit (qmax = 7, W4A4) or
+// 3-bit (qmax = 3, W3A3) activation quantization (zh §3-§4, fr §4). Since
+// |h'| <= amax, |fl(h' * fl(qmax/amax))| <= qmax (1+2^-24)^2 < qmax + 0.5, so
+// the code is always in [-qmax, qmax] and no clamp is needed.
 //
 // Cluster design (B200): a tile of T tokens is split along D over a
 // thread-block cluster of C CTAs (one per SM); CTA c owns the columns
@@ -62,10 +63,11 @@ __device__ __forceinline__ uint32_t quantize8(const uint4 hv, float inv) {
   return packed;
 }
 
-__device__ __forceinline__ void inv_and_scale(float amax, float& inv, float& scale) {
+// qmax = 7 (INT4 codes) or 3 (INT3 codes, W3A3).
+__device__ __forceinline__ void inv_and_scale(float amax, float qmax, float& inv, float& scale) {
   if (amax >= kZeroTokenAmax) {
-    inv = __fdiv_rn(7.0f, amax);
-    scale = __fdiv_rn(amax, 7.0f);
+    inv = __fdiv_rn(qmax, amax);
+    scale = __fdiv_rn(amax, qmax);
   } else {
     inv = 0.0f;
     scale = 0.0f;
@@ -172,7 +174,7 @@ __device__ __forceinline__ void publish_amax(float (&rmax)[MT][2], float* wamax,
 template <int T>
 __device__ __forceinline__ void gather_amax(uint32_t amaxbuf_addr, float* am2, float* rowinv,
                                             float* scale_out, uint32_t csize, uint32_t crank,
-                                            int row0, int N, int tid) {
+                                            int row0, int N, int tid, float qmax) {
   for (int i = tid; i < static_cast<int>(csize) * T; i += kBoundaryThreads) {
     const uint32_t c = static_cast<uint32_t>(i / T);
     am2[i] = ld_dsmem_f32(map_to_rank(amaxbuf_addr + 4u * (i % T), c));
@@ -182,7 +184,7 @@ __device__ __forceinline__ void gather_amax(uint32_t amaxbuf_addr, float* am2, f
     float m = 0.f;
     for (uint32_t c = 0; c < csize; ++c) m = fmaxf(m, am2[c * T + tid]);
     float inv, sc;
-    inv_and_scale(m, inv, sc);
+    inv_and_scale(m, qmax, inv, sc);
     rowinv[tid] = inv;
     if (crank == 0 && row0 + tid < N) scale_out[row0 + tid] = sc;
   }
@@ -269,7 +271,7 @@ __global__ void __launch_bounds__(kRfThreads, 1)
 boundary_cluster_rf_kernel(const bf16* __restrict__ x, const bf16* __restrict__ res,
                            const uint4* __restrict__ Uf, const uint4* __restrict__ Vf, int N,
                            int D, void* __restrict__ h_out, uint8_t* __restrict__ q_out,
-                           float* __restrict__ scale_out) {
+                           float* __restrict__ scale_out, float qmax) {
   using C = RfCfg<R, T, Dc>;
   constexpr int S = C::S, RP = C::RP;
   constexpr uint32_t pitch = C::pitch;
@@ -501,7 +503,7 @@ boundary_cluster_rf_kernel(const bf16* __restrict__ x, const bf16* __restrict__ 
       float m = 0.f;
       for (uint32_t c = 0; c < csize; ++c) m = fmaxf(m, am2[c * T + tid]);
       float inv, sc;
-      inv_and_scale(m, inv, sc);
+      inv_and_scale(m, qmax, inv, sc);
       rowinv[tid] = inv;
       if (crank == 0 && row0 + tid < N) scale_out[row0 + tid] = sc;
     }
@@ -592,7 +594,7 @@ boundary_cluster_smem_kernel(const bf16* __restrict__ x, const bf16* __restrict_
                              const bf16* __restrict__ Ut,   // [R, D]  (U transposed, zero padded)
                              const bf16* __restrict__ V,    // [D, R]  (zero padded)
                              int N, int D, int Dc, void* __restrict__ h_out,
-                             uint8_t* __restrict__ q_out, float* __restrict__ scale_out) {
+                             uint8_t* __restrict__ q_out, float* __restrict__ scale_out, float qmax) {
   using C = SmemCfg<T, R>;
   constexpr int RP = C::RP;
   extern __shared__ __align__(128) uint8_t smem[];
@@ -791,7 +793,7 @@ boundary_cluster_smem_kernel(const bf16* __restrict__ x, const bf16* __restrict_
 
     // ---- amax over the cluster, then codes
     cluster_sync();
-    gather_amax<T>(sbase + L.amaxbuf, am2, rowinv, scale_out, csize, crank, row0, N, tid);
+    gather_amax<T>(sbase + L.amaxbuf, am2, rowinv, scale_out, csize, crank, row0, N, tid, qmax);
     store_tile<F32OUT>(xs_ptr, pitch, rowinv, T, Dc, row0, N, D, col0, h_out, q_out, tid);
     fence_proxy_async_smem();
     __syncthreads();
@@ -805,7 +807,7 @@ template <int THREADS, bool F32OUT>
 __global__ void __launch_bounds__(THREADS)
 boundary_rowwise_kernel(const bf16* __restrict__ x, const bf16* __restrict__ res, int N, int D,
                         void* __restrict__ h_out, uint8_t* __restrict__ q_out,
-                        float* __restrict__ scale_out) {
+                        float* __restrict__ scale_out, float qmax) {
   constexpr int VPT = 8;  // 16-byte vectors per thread (D <= THREADS * 64)
   __shared__ float red[THREADS / 32];
   __shared__ float s_inv;
@@ -850,7 +852,7 @@ boundary_rowwise_kernel(const bf16* __restrict__ x, const bf16* __restrict__ res
       float m = 0.f;
       for (int w = 0; w < THREADS / 32; ++w) m = fmaxf(m, red[w]);
       float inv, sc;
-      inv_and_scale(m, inv, sc);
+      inv_and_scale(m, qmax, inv, sc);
       s_inv = inv;
       scale_out[row] = sc;
     }

@@ -5,7 +5,7 @@
 // ReSpinQuant explainers, zh §2.2 steps 1-3, row convention, then W4A4
 // activation quantization, zh §3-§4):
 //   y = residual U ;  h = (residual + x) + y V^T  (fp32) ;  h' = bf16(h)
-//   amax = max|h'| ; inv = 7/amax ; q = rint(h' inv)
+//   amax = max|h'| ; inv = qmax/amax ; q = rint(h' inv)   (qmax = 7 or 3)
 //
 // Design (one CTA per SM, persistent over 16-token tiles, no cluster):
 //  * the residual tile (16 x D bf16) is brought into shared memory by 2-D
@@ -141,7 +141,7 @@ __global__ void __launch_bounds__(32 * W, 1)
 boundary_rowtile_kernel(const __grid_constant__ CUtensorMap tmR, const __grid_constant__ CUtensorMap tmX,
                         const uint4* __restrict__ Ut,
                         const uint4* __restrict__ Vt, int N, void* __restrict__ h_out,
-                        uint8_t* __restrict__ q_out, float* __restrict__ scale_out) {
+                        uint8_t* __restrict__ q_out, float* __restrict__ scale_out, float qmax) {
   using C = RtCfg<R, W>;
   constexpr int XS = C::XS, RING = C::RING, D = NB * 64 * W;
   extern __shared__ uint8_t smem_raw[];
@@ -366,7 +366,7 @@ boundary_rowtile_kernel(const __grid_constant__ CUtensorMap tmR, const __grid_co
 #pragma unroll
       for (int w = 0; w < W; ++w) m = fmaxf(m, wamax[w * kRtT + tid]);
       float inv, sc;
-      inv_and_scale(m, inv, sc);
+      inv_and_scale(m, qmax, inv, sc);
       rowinv[tid] = inv;
       if (row0 + tid < N) scale_out[row0 + tid] = sc;
     }

@@ -366,7 +366,8 @@ respin_status_t respin_plan_create(respin_plan_t* out, int D, int r, const float
     return fail(RESPIN_ERR_UNSUPPORTED, "r=%d: need 0 <= r <= 128 and r %% 8 == 0", r);
   if (r > 0 && (U_r == nullptr || V_r == nullptr))
     return fail(RESPIN_ERR_INVALID_ARG, "U_r and V_r must be non-NULL when r > 0");
-  if (flags & ~RESPIN_H_FP32_DEBUG) return fail(RESPIN_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
+  if (flags & ~(RESPIN_H_FP32_DEBUG | RESPIN_ACT_INT3))
+    return fail(RESPIN_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
   const int r_pad = r == 0 ? 0 : (r <= 16 ? 16 : r <= 32 ? 32 : r <= 64 ? 64 : 128);
   if (fault_at("plan_alloc")) return fail(RESPIN_ERR_OOM, "injected fault at plan_alloc");
 
@@ -481,6 +482,7 @@ respin_status_t respin_boundary_forward(respin_plan_t plan, const void* x, const
 
   const int D = plan->D;
   const bool f32 = (plan->flags & RESPIN_H_FP32_DEBUG) != 0;
+  float qmax = (plan->flags & RESPIN_ACT_INT3) != 0 ? 3.0f : 7.0f;   // largest code magnitude
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bf16* xb = static_cast<const bf16*>(x);
   const bf16* rb = static_cast<const bf16*>(residual);
@@ -490,11 +492,11 @@ respin_status_t respin_boundary_forward(respin_plan_t plan, const void* x, const
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, plan->device);
     const int grid = N < sms * 16 ? N : sms * 16;
     if (D <= 256 * 64) {
-      if (f32) boundary_rowwise_kernel<256, true><<<grid, 256, 0, s>>>(xb, rb, N, D, h_out, q_packed, scale);
-      else boundary_rowwise_kernel<256, false><<<grid, 256, 0, s>>>(xb, rb, N, D, h_out, q_packed, scale);
+      if (f32) boundary_rowwise_kernel<256, true><<<grid, 256, 0, s>>>(xb, rb, N, D, h_out, q_packed, scale, qmax);
+      else boundary_rowwise_kernel<256, false><<<grid, 256, 0, s>>>(xb, rb, N, D, h_out, q_packed, scale, qmax);
     } else {
-      if (f32) boundary_rowwise_kernel<1024, true><<<grid, 1024, 0, s>>>(xb, rb, N, D, h_out, q_packed, scale);
-      else boundary_rowwise_kernel<1024, false><<<grid, 1024, 0, s>>>(xb, rb, N, D, h_out, q_packed, scale);
+      if (f32) boundary_rowwise_kernel<1024, true><<<grid, 1024, 0, s>>>(xb, rb, N, D, h_out, q_packed, scale, qmax);
+      else boundary_rowwise_kernel<1024, false><<<grid, 1024, 0, s>>>(xb, rb, N, D, h_out, q_packed, scale, qmax);
     }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "boundary_rowwise_kernel launch");
@@ -512,7 +514,7 @@ respin_status_t respin_boundary_forward(respin_plan_t plan, const void* x, const
     const uint4* ut = reinterpret_cast<const uint4*>(fac);
     const uint4* vt = reinterpret_cast<const uint4*>(fac + static_cast<size_t>(plan->r_pad) * D);
     const int grid = ntiles < c.max_clusters ? ntiles : c.max_clusters;
-    void* args[] = {&tmR, &tmX, &ut, &vt, &N, &h_out, &q_packed, &scale};
+    void* args[] = {&tmR, &tmX, &ut, &vt, &N, &h_out, &q_packed, &scale, &qmax};
     cudaError_t e = cudaLaunchKernel(c.fn, dim3(grid), dim3(32 * c.cluster), args, c.smem, s);
     if (e != cudaSuccess) return cuda_fail(e, "boundary_rowtile_kernel launch");
     return ok();
@@ -534,13 +536,13 @@ respin_status_t respin_boundary_forward(respin_plan_t plan, const void* x, const
   if (c.rf) {
     const uint4* uf = reinterpret_cast<const uint4*>(fac);
     const uint4* vf = reinterpret_cast<const uint4*>(fac + static_cast<size_t>(plan->r_pad) * D);
-    void* args[] = {&xb, &rb, &uf, &vf, &N, const_cast<int*>(&D), &h_out, &q_packed, &scale};
+    void* args[] = {&xb, &rb, &uf, &vf, &N, const_cast<int*>(&D), &h_out, &q_packed, &scale, &qmax};
     e = cudaLaunchKernelExC(&lc, c.fn, args);
   } else {
     const bf16* ut = fac;
     const bf16* v = fac + static_cast<size_t>(plan->r_pad) * D;
     int Dc = c.Dc;
-    void* args[] = {&xb, &rb, &ut, &v, &N, const_cast<int*>(&D), &Dc, &h_out, &q_packed, &scale};
+    void* args[] = {&xb, &rb, &ut, &v, &N, const_cast<int*>(&D), &Dc, &h_out, &q_packed, &scale, &qmax};
     e = cudaLaunchKernelExC(&lc, c.fn, args);
   }
   if (e != cudaSuccess) return cuda_fail(e, "boundary_cluster_kernel launch");

@@ -23,10 +23,11 @@ def bf16_keys(bits: np.ndarray) -> np.ndarray:
 
 
 def run_boundary(fx: W.BoundaryFixture, *, f32: bool, residual=True,
-                 h_out=True, device="cuda"):
-    """Run respin_boundary_forward on the fixture; returns numpy results."""
+                 h_out=True, device="cuda", qmax=7):
+    """Run respin_boundary_forward on the fixture (INT4 codes, or INT3 codes
+    for qmax = 3); returns numpy results."""
     D, N, r = fx.D, fx.N, fx.r
-    flags = rq.RESPIN_H_FP32_DEBUG if f32 else 0
+    flags = (rq.RESPIN_H_FP32_DEBUG if f32 else 0) | (rq.RESPIN_ACT_INT3 if qmax == 3 else 0)
     U32 = fx.U.astype(np.float32) if r else None
     V32 = fx.V.astype(np.float32) if r else None
     plan = rq.Plan(D, r, U32, V32, flags)
@@ -49,7 +50,7 @@ def run_boundary(fx: W.BoundaryFixture, *, f32: bool, residual=True,
     return out
 
 
-def oracle_boundary(fx: W.BoundaryFixture, rows=None, residual=True):
+def oracle_boundary(fx: W.BoundaryFixture, rows=None, residual=True, qmax=7):
     """Oracle for the fixture (optionally a row subset)."""
     x = fx.x.float().numpy()
     res = fx.residual.float().numpy() if residual else None
@@ -58,7 +59,7 @@ def oracle_boundary(fx: W.BoundaryFixture, rows=None, residual=True):
         res = res[rows] if res is not None else None
     U32 = fx.U.astype(np.float32)
     V32 = fx.V.astype(np.float32)
-    return O.boundary_reference(x, res, U32, V32)
+    return O.boundary_reference(x, res, U32, V32, qmax)
 
 
 def check_h_f32(h_gpu: np.ndarray, h64: np.ndarray) -> float:
@@ -105,9 +106,9 @@ def check_bf16_output(h_bits: np.ndarray, h64: np.ndarray) -> float:
     return worst
 
 
-def check_codes_on_own_h(h_bits, q_packed, scale):
+def check_codes_on_own_h(h_bits, q_packed, scale, qmax=7):
     """Codes and scales bit-exact vs the oracle quantizer on the GPU's h'."""
-    codes, sc = O.quantize_int4_per_token(O.bf16_bits_to_f32(h_bits))
+    codes, sc = O.quantize_per_token(O.bf16_bits_to_f32(h_bits), qmax)
     assert np.array_equal(scale.view(np.uint32), sc.view(np.uint32)), \
         "scales differ"
     assert np.array_equal(q_packed, O.pack_int4(codes)), "codes differ"

@@ -33,6 +33,13 @@ def test_header_symbols_exported():
         assert hasattr(rq.lib, n), n
 
 
+def test_header_flag_values_match_binding():
+    src = open(HEADER).read()
+    flags = dict((m, int(v)) for m, v in re.findall(r"#define (RESPIN_\w+) (\d+)u", src))
+    assert flags == {"RESPIN_H_FP32_DEBUG": rq.RESPIN_H_FP32_DEBUG,
+                     "RESPIN_ACT_INT3": rq.RESPIN_ACT_INT3}
+
+
 def test_version():
     assert "sm_100a" in rq.version()
 

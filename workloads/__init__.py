@@ -252,6 +252,18 @@ def int4_packed_random(rows: int, K: int, seed: int = 0,
                                          dtype=np.uint8)
 
 
+def int3_packed_random(rows: int, K: int, seed: int = 0,
+                       tensor_id: int = TID_WEIGHTS) -> np.ndarray:
+    """uint8 [rows, K/2]: two uniformly random 3-bit codes (-4..3) per byte,
+    each in a two's-complement nibble (low nibble first)."""
+    b = int4_packed_random(rows, K, seed, tensor_id)
+    lo, hi = b & 7, (b >> 4) & 7
+    # 3-bit two's complement -> 4-bit: copy bit 2 into bit 3
+    lo = lo | ((lo & 4) << 1)
+    hi = hi | ((hi & 4) << 1)
+    return (lo | (hi << 4)).astype(np.uint8)
+
+
 def weight_scales(O: int, K: int, seed: int = 0) -> np.ndarray:
     """float32 [O] per-output-channel scales U(0.5, 1.5) / (4.61 sqrt(K))."""
     u = rng(seed, TID_WSCALE).uniform(0.5, 1.5, size=O)
