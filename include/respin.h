@@ -58,10 +58,11 @@ typedef struct respin_plan_s* respin_plan_t;
 #define RESPIN_H_FP32_DEBUG 1u
 
 /* Plan flag: 3-bit activation codes (W3A3, named beside W4A4 on the
- * explainer pages: zh §3-§4, it §3, nl §3, fr §4; no quantizer is given
- * there). The quantizer bound becomes 3 instead of 7: inv = 3 / amax,
- * scale = amax / 3, codes in [-3, 3], stored in the same two's-complement
- * nibbles, so w4a4_gemm consumes them (and 3-bit weight codes) unchanged. */
+ * explainer pages: zh §3-§4, it §3-§4, nl §3-§4, es §3-§4, fr §4; no
+ * quantizer is given there). The quantizer bound becomes 3 instead of 7:
+ * inv = 3 / amax, scale = amax / 3, codes in [-3, 3], stored in the same
+ * two's-complement nibbles, so w4a4_gemm consumes them (and 3-bit weight
+ * codes) unchanged. */
 #define RESPIN_ACT_INT3 2u
 
 /*

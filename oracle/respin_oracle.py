@@ -30,9 +30,9 @@ What the pages fix, and how this module follows it:
   all in IEEE binary32, on the bfloat16-rounded boundary output ``g``. Tokens
   with ``amax < 2^-125`` get scale 0 and all-zero codes (below that
   ``7 / amax`` would overflow binary32).
-* 3-bit activations (W3A3, named beside W4A4 in zh §3-§4, it §3, nl §3 and
-  fr §4; no quantizer given either). Reading: the same per-token symmetric
-  form with bound 3 instead of 7: ``inv = 3 / amax``,
+* 3-bit activations (W3A3, named beside W4A4 in zh §3-§4, it §3-§4,
+  nl §3-§4, es §3-§4 and fr §4; no quantizer given either). Reading: the same
+  per-token symmetric form with bound 3 instead of 7: ``inv = 3 / amax``,
   ``q = clamp(rint(g * inv), -4, 3)``, ``scale = amax / 3``; codes stay in
   4-bit containers (the pages give no 3-bit packing), so the integer GEMM is
   the same for both widths.

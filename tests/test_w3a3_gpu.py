@@ -1,10 +1,10 @@
 """GPU parity of the W3A3 path (3-bit activation codes) against the oracle.
 
 W3A3 is the second quantization setting the ReSpinQuant explainers report
-beside W4A4 (zh §3-§4, it §3, nl §3, fr §4); the pages give no quantizer for
-either. Reading (same as the oracle's): the per-token symmetric quantizer with
-bound 3 (inv = 3/amax, scale = amax/3, codes in [-3, 3]) in the same nibble
-containers, so the integer GEMM is unchanged. Every boundary kernel family is
+beside W4A4 (zh §3-§4, it §3-§4, nl §3-§4, es §3-§4, fr §4); the pages give
+no quantizer for either. Reading (same as the oracle's): the per-token
+symmetric quantizer with bound 3 (inv = 3/amax, scale = amax/3, codes in
+[-3, 3]) in the same nibble containers, so the integer GEMM is unchanged. Every boundary kernel family is
 run with the RESPIN_ACT_INT3 plan flag; the codes feed the W4A4 GEMM with
 3-bit weights.
 """
