@@ -275,10 +275,17 @@ boundary_rowtile_kernel(const __grid_constant__ CUtensorMap tmR, const __grid_co
       split_bf16x2(y3, ahi[kk][3], alo[kk][3]);
     }
     uint32_t amax2[2] = {0u, 0u};   // running max |h'| (bf16x2) of rows g and g + 8
-    // (row, chunk t) -> row * 128 + ((t ^ row % 8) << 4): the XOR only touches
-    // bits 4-6, which are zero in row * 128 + 4 q4, so it folds into one XOR.
-    const uint32_t rb[2] = {static_cast<uint32_t>(g * 128 + 4 * q4 + (g << 4)),
-                            static_cast<uint32_t>((g + 8) * 128 + 4 * q4 + (g << 4))};
+    // The plan orders V so that n8 tile t of a block holds columns
+    // 16 (n / 2) + 2 t + n % 2 (n = 0..7 the tile's column index): this lane's
+    // accumulators are then columns 16 q4 .. 16 q4 + 15, i.e. the 16-byte
+    // chunks 2 q4 (tiles 0-3) and 2 q4 + 1 (tiles 4-7) of rows g and g + 8,
+    // at row * 128 + ((chunk ^ row % 8) << 4) (row % 8 = g for both rows).
+    uint32_t cb[2][2];
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+      for (int half = 0; half < 2; ++half)
+        cb[hh][half] = static_cast<uint32_t>((g + 8 * hh) * 128 + (((2 * q4 + half) ^ g) << 4));
 #pragma unroll
     for (int j = 0; j < NB; ++j) {
       if (j + RING - 1 < NB) load_v(vb[(j + RING - 1) % RING], j + RING - 1);
@@ -308,41 +315,43 @@ boundary_rowtile_kernel(const __grid_constant__ CUtensorMap tmR, const __grid_co
           mma_bf16_16816(acc[t], alo[kk], u4c(v, ri % 4), u4c(v, ri % 4 + 1));
         }
       }
-      // All loads of the block first, then the arithmetic, then the stores:
-      // h' overwrites the residual in place at XOR-computed offsets, which
-      // the compiler cannot prove distinct, so interleaved loads and stores
-      // would serialise the 16 pairs of a lane into one dependency chain.
-      uint32_t rw[8][2], xw[8][2];
+      // All loads of the block first (four 16-byte chunks of residual and
+      // of x), then the arithmetic, then the in-place h' stores.
+      uint32_t rw[2][2][4], xw[2][2][4];   // [hh][half][word]: word i = tile 4 half + i
 #pragma unroll
-      for (int t = 0; t < 8; ++t)
+      for (int hh = 0; hh < 2; ++hh)
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          const uint32_t off = rb[hh] ^ static_cast<uint32_t>(t << 4);
-          rw[t][hh] = *reinterpret_cast<const uint32_t*>(blk + off);
-          xw[t][hh] = *reinterpret_cast<const uint32_t*>(xblk + off);
+        for (int half = 0; half < 2; ++half) {
+          const uint4 rv = *reinterpret_cast<const uint4*>(blk + cb[hh][half]);
+          const uint4 xv = *reinterpret_cast<const uint4*>(xblk + cb[hh][half]);
+          rw[hh][half][0] = rv.x; rw[hh][half][1] = rv.y; rw[hh][half][2] = rv.z; rw[hh][half][3] = rv.w;
+          xw[hh][half][0] = xv.x; xw[hh][half][1] = xv.y; xw[hh][half][2] = xv.z; xw[hh][half][3] = xv.w;
         }
 #pragma unroll
-      for (int t = 0; t < 8; ++t) {
+      for (int hh = 0; hh < 2; ++hh)
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          const float2 sum = add_f32x2(bf16x2_to_f32x2(rw[t][hh]), bf16x2_to_f32x2(xw[t][hh]));
-          const float2 h = add_f32x2(sum, make_float2(acc[t][2 * hh], acc[t][2 * hh + 1]));
-          const uint32_t hb = pack_bf16x2(h.x, h.y);
-          rw[t][hh] = hb;
-          amax2[hh] = absmax_bf16x2(amax2[hh], hb);
-          if constexpr (F32OUT) {
-            const int row = g + 8 * hh;
-            if (h_out != nullptr && row0 + row < N)
-              *reinterpret_cast<float2*>(static_cast<float*>(h_out) + static_cast<size_t>(row0 + row) * D +
-                                         colb + 8 * t + 2 * q4) = h;
+        for (int half = 0; half < 2; ++half)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int t = 4 * half + i;
+            const float2 sum = add_f32x2(bf16x2_to_f32x2(rw[hh][half][i]), bf16x2_to_f32x2(xw[hh][half][i]));
+            const float2 h = add_f32x2(sum, make_float2(acc[t][2 * hh], acc[t][2 * hh + 1]));
+            const uint32_t hb = pack_bf16x2(h.x, h.y);
+            rw[hh][half][i] = hb;
+            amax2[hh] = absmax_bf16x2(amax2[hh], hb);
+            if constexpr (F32OUT) {
+              const int row = g + 8 * hh;
+              if (h_out != nullptr && row0 + row < N)
+                *reinterpret_cast<float2*>(static_cast<float*>(h_out) + static_cast<size_t>(row0 + row) * D +
+                                           colb + 16 * q4 + 2 * t) = h;
+            }
           }
-        }
-      }
 #pragma unroll
-      for (int t = 0; t < 8; ++t)
+      for (int hh = 0; hh < 2; ++hh)
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh)
-          *reinterpret_cast<uint32_t*>(blk + (rb[hh] ^ static_cast<uint32_t>(t << 4))) = rw[t][hh];
+        for (int half = 0; half < 2; ++half)
+          *reinterpret_cast<uint4*>(blk + cb[hh][half]) =
+              make_uint4(rw[hh][half][0], rw[hh][half][1], rw[hh][half][2], rw[hh][half][3]);
       // the slot's bytes were read (generic proxy) before its next tensor copy
       fence_proxy_async_smem();
       __syncwarp();
@@ -400,8 +409,9 @@ boundary_rowtile_kernel(const __grid_constant__ CUtensorMap tmR, const __grid_co
 // (U[d][n], U[d+1][n]) with d = 64 b + 16 kk + 2q + 8e, n = 8p + g, stored at
 // uint4 ((b 4 + kk) R/16 + i/4) * 32 + lane, component i % 4. Vt: for block b,
 // register i = 2 (t R/16 + kk) + e holds (V[d][m], V[d][m+1]) with
-// d = 64 b + 8t + g, m = 16 kk + 2q + 8e, stored at uint4 (b R/4 + i/4) * 32 +
-// lane, component i % 4.
+// d = 64 b + 16 (g / 2) + 2 t + g % 2 (the column order that gives each lane
+// 16 contiguous output columns), m = 16 kk + 2q + 8e, stored at uint4
+// (b R/4 + i/4) * 32 + lane, component i % 4.
 inline void rt_pack_factors(const uint16_t* Ub, const uint16_t* Vb, int D, int R, uint32_t* Ut, uint32_t* Vt) {
   auto pair = [](uint16_t lo, uint16_t hi) { return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16); };
   const int UQ = R / 16, KK = R / 16, VB = R / 4;
@@ -417,7 +427,7 @@ inline void rt_pack_factors(const uint16_t* Ub, const uint16_t* Vb, int D, int R
         }
       for (int i = 0; i < 4 * VB; ++i) {
         const int e = i % 2, tk = i / 2, kk = tk % KK, t = tk / KK;
-        const int d = 64 * b + 8 * t + g, m = 16 * kk + 2 * q + 8 * e;
+        const int d = 64 * b + 16 * (g >> 1) + 2 * t + (g & 1), m = 16 * kk + 2 * q + 8 * e;
         const size_t idx = ((static_cast<size_t>(b) * VB + i / 4) * 32 + lane) * 4 + i % 4;
         Vt[idx] = pair(Vb[static_cast<size_t>(d) * R + m], Vb[static_cast<size_t>(d) * R + m + 1]);
       }
