@@ -87,12 +87,23 @@ struct respin_plan_s {
   bool has_small = false;
   __nv_bfloat16* factors_small = nullptr;
   BoundaryConfig cfg_small;
+  // Third configuration for the fewest tokens: 8-CTA instead of 4-CTA
+  // clusters (each SM pulls half the factor bytes of a tile from L2).
+  bool has_tiny = false;
+  __nv_bfloat16* factors_tiny = nullptr;
+  BoundaryConfig cfg_tiny;
 };
 
 // Calls with at most this many tokens use cfg_small when the plan has one
 // (row tiles: one 16-token tile per SM; a 4-CTA cluster tile chain is about a
 // third as long, so clusters win until their tile rounds add up).
 constexpr int kSmallTokens = 1280;
+// Calls with at most this many tokens (and no more tiles than co-resident
+// 8-CTA clusters) use cfg_tiny. Measured on B200, D = 4096, r = 32, CUDA-graph
+// replay, 4- vs 8-CTA clusters: N = 1: 6.7 vs 5.5 us, 8: 7.2 vs 6.2 us,
+// 64: 7.8 vs 6.8 us; at 256 tokens (16 tiles) the 8-CTA clusters take two
+// rounds: 7.8 vs 11.6 us.
+constexpr int kTinyTokens = 128;
 
 namespace {
 
@@ -242,7 +253,10 @@ int max_active_clusters(const void* fn, int C, size_t smem, int threads) {
 // Choose the boundary kernel. r <= 32: register-resident factors with 512
 // (else 256) columns per CTA. Otherwise: shared-memory factors, the smallest
 // cluster whose per-CTA slice fits, preferring 32-token tiles.
-respin_status_t configure_boundary(int D, int R, bool f32, BoundaryConfig* out, bool allow_rowtile = true) {
+// only_dc > 0: the register-factor cluster kernel with that column slice, or
+// UNSUPPORTED.
+respin_status_t configure_boundary(int D, int R, bool f32, BoundaryConfig* out, bool allow_rowtile = true,
+                                   int only_dc = 0) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
@@ -266,7 +280,7 @@ respin_status_t configure_boundary(int D, int R, bool f32, BoundaryConfig* out, 
   }
   if (R <= 32) {
     for (int Dc : {1024, 512, 256}) {
-      if (D % Dc || D / Dc > 16) continue;
+      if (D % Dc || D / Dc > 16 || (only_dc > 0 && Dc != only_dc)) continue;
       const int C = D / Dc;
       const size_t smem = rf_smem(R, Dc);
       if (smem == 0 || smem > static_cast<size_t>(smem_optin)) continue;
@@ -278,6 +292,7 @@ respin_status_t configure_boundary(int D, int R, bool f32, BoundaryConfig* out, 
       return ok();
     }
   }
+  if (only_dc > 0) return fail(RESPIN_ERR_UNSUPPORTED, "no register-factor configuration with Dc=%d", only_dc);
   // Shared-memory factor slices (both, else U^T only with V read from L2).
   for (bool vres : {true, false}) {
     for (int C : {1, 2, 4, 8, 16}) {
@@ -425,10 +440,17 @@ respin_status_t respin_plan_create(respin_plan_t* out, int D, int r, const float
       st2 = upload(p->cfg_small, &p->factors_small);
       p->has_small = st2 == RESPIN_OK;
     }
+    if (st2 == RESPIN_OK && p->has_small && p->cfg_small.rf && p->cfg_small.cluster == 4 &&
+        configure_boundary(D, r_pad, (flags & RESPIN_H_FP32_DEBUG) != 0, &p->cfg_tiny, false, 512) == RESPIN_OK &&
+        p->cfg_tiny.cluster == 8) {
+      st2 = upload(p->cfg_tiny, &p->factors_tiny);
+      p->has_tiny = st2 == RESPIN_OK;
+    }
     t_last_error.clear();
     if (st2 != RESPIN_OK || p->factors == nullptr) {
       if (p->factors) cudaFree(p->factors);
       if (p->factors_small) cudaFree(p->factors_small);
+      if (p->factors_tiny) cudaFree(p->factors_tiny);
       delete p;
       return st2 != RESPIN_OK ? st2 : fail(RESPIN_ERR_OOM, "factor upload failed");
     }
@@ -457,6 +479,7 @@ respin_status_t respin_plan_destroy(respin_plan_t plan) {
     cudaError_t e = cudaDeviceSynchronize();
     if (e == cudaSuccess) e = cudaFree(plan->factors);
     if (e == cudaSuccess && plan->factors_small) e = cudaFree(plan->factors_small);
+    if (e == cudaSuccess && plan->factors_tiny) e = cudaFree(plan->factors_tiny);
     if (e != cudaSuccess) st = cuda_fail(e, "releasing plan factors");
     cudaSetDevice(cur);
   }
@@ -503,9 +526,10 @@ respin_status_t respin_boundary_forward(respin_plan_t plan, const void* x, const
     return ok();
   }
 
-  const bool small = plan->has_small && N <= kSmallTokens;
-  const BoundaryConfig& c = small ? plan->cfg_small : plan->cfg;
-  const bf16* fac = small ? plan->factors_small : plan->factors;
+  const bool tiny = plan->has_tiny && N <= kTinyTokens && (N + kRfT - 1) / kRfT <= plan->cfg_tiny.max_clusters;
+  const bool small = !tiny && plan->has_small && N <= kSmallTokens;
+  const BoundaryConfig& c = tiny ? plan->cfg_tiny : small ? plan->cfg_small : plan->cfg;
+  const bf16* fac = tiny ? plan->factors_tiny : small ? plan->factors_small : plan->factors;
   const int ntiles = (N + c.T - 1) / c.T;
   if (c.kind == kRowTile) {
     CUtensorMap tmR, tmX;
