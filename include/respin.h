@@ -158,6 +158,51 @@ respin_status_t w4a4_gemm_i32(const uint8_t* q_act, const uint8_t* q_w,
                               int N, int K, int O, int32_t* acc_out,
                               void* stream);
 
+/*
+ * respin_factors_from_subspace -- plan factors from the subspace form.
+ *
+ * Passage: zh §2.2 steps 1-3 store one D x r basis Q and an r x r rotation
+ * R_sub per boundary and apply x + Q ((R_sub - I) (Q^T x)) to a column
+ * vector. For a row vector h the same map is h + (h U_r) V_r^T with
+ *     U_r = Q,   V_r = Q (R_sub - I)
+ * (computed in float64, rounded to float).
+ *
+ *   D, r   : 0 < r <= D.
+ *   Q      : HOST fp32 [D, r] row-major.
+ *   R_sub  : HOST fp32 [r, r] row-major.
+ *   U_r    : HOST fp32 [D, r] output (caller-owned).
+ *   V_r    : HOST fp32 [D, r] output (caller-owned).
+ * Host only (no device, no allocation). Errors: INVALID_ARG.
+ */
+respin_status_t respin_factors_from_subspace(int D, int r, const float* Q,
+                                            const float* R_sub, float* U_r,
+                                            float* V_r);
+
+/*
+ * respin_factors_from_transition -- plan factors from a dense transition.
+ *
+ * Passage: the top-r SVD of Delta T = T - I gives the subspace (it §2C,
+ * nl §2C, es §2B, fr §2C). Row convention h' = h T: with
+ * Delta T = sum_i s_i u_i v_i^T (s_1 >= s_2 >= ...),
+ *     U_r = [u_1 .. u_r],   V_r = [s_1 v_1 .. s_r v_r],
+ * so h (I + U_r V_r^T) is the best rank-r fix in the Frobenius norm. Float64
+ * block subspace iteration (block max(2r, r + 8), deterministic start) with
+ * Rayleigh-Ritz steps until the top-r subspace stops moving.
+ *
+ *   D, r    : 0 < r < D, r <= 128.
+ *   T       : HOST fp32 [D, D] row-major.
+ *   gap_tol : the truncation is refused (UNSUPPORTED) unless
+ *             s_r - s_(r+1) > gap_tol * s_1; without a gap the top-r subspace
+ *             is not unique (e.g. r splitting a pair of equal singular values).
+ *   U_r,V_r : HOST fp32 [D, r] outputs (caller-owned).
+ *   sigma   : HOST fp64 [r + 1] output s_1 .. s_(r+1), or NULL. Also written
+ *             when the gap check refuses.
+ * Host only; O(D^2 r) work per iteration. Errors: INVALID_ARG, UNSUPPORTED.
+ */
+respin_status_t respin_factors_from_transition(int D, int r, const float* T,
+                                               double gap_tol, float* U_r,
+                                               float* V_r, double* sigma);
+
 /* respin_device_status -- synchronizes the current device, then returns and
  * clears the device status word through *code (0 = no kernel gave up; else
  * the site that gave up). Returns DEVICE_CHECK if *code != 0. */

@@ -28,6 +28,7 @@ RESPIN_ACT_INT3 = 2
 # Every entry point include/respin.h declares (checked by the tests).
 EXPORTED = ("respin_plan_create", "respin_plan_destroy",
             "respin_boundary_forward", "w4a4_gemm", "w4a4_gemm_i32",
+            "respin_factors_from_subspace", "respin_factors_from_transition",
             "respin_device_status", "respin_last_error", "respin_version")
 
 
@@ -44,7 +45,7 @@ def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(
             f"{LIB_PATH} is missing: build it with "
-            "`python -m rotation_post_quantization_b200.build`")
+            "`python rotation_post_quantization_b200/build.py`")
     lib = ctypes.CDLL(LIB_PATH)
     vp, i32, u32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_uint
     fp = ctypes.POINTER(ctypes.c_float)
@@ -53,6 +54,9 @@ def _load() -> ctypes.CDLL:
     lib.respin_boundary_forward.argtypes = [vp, vp, vp, i32, vp, vp, vp, vp]
     lib.w4a4_gemm.argtypes = [vp, vp, vp, vp, i32, i32, i32, vp, vp]
     lib.w4a4_gemm_i32.argtypes = [vp, vp, i32, i32, i32, vp, vp]
+    dp = ctypes.POINTER(ctypes.c_double)
+    lib.respin_factors_from_subspace.argtypes = [i32, i32, fp, fp, fp, fp]
+    lib.respin_factors_from_transition.argtypes = [i32, i32, fp, ctypes.c_double, fp, fp, dp]
     lib.respin_device_status.argtypes = [ctypes.POINTER(ctypes.c_int)]
     for name in EXPORTED[:-2]:
         getattr(lib, name).restype = ctypes.c_int
@@ -158,6 +162,45 @@ def w4a4_gemm_i32(q_act, q_w, acc_out, stream=None) -> None:
     O = q_w.shape[0]
     _check(lib.w4a4_gemm_i32(_ptr(q_act), _ptr(q_w), int(N), int(2 * K2),
                              int(O), _ptr(acc_out), _stream(stream)))
+
+
+def _host_f32(a, shape, name):
+    a = np.ascontiguousarray(a, dtype=np.float32)
+    if a.shape != shape:
+        raise ValueError(f"{name} must have shape {shape}")
+    return a
+
+
+def respin_factors_from_subspace(Q, R_sub):
+    """(U_r, V_r) = (Q, Q (R_sub - I)) for the plan, from the subspace form
+    (host fp32 arrays Q [D, r] and R_sub [r, r])."""
+    Q = np.ascontiguousarray(Q, dtype=np.float32)
+    D, r = Q.shape
+    R = _host_f32(R_sub, (r, r), "R_sub")
+    fp = ctypes.POINTER(ctypes.c_float)
+    U = np.empty((D, r), np.float32)
+    V = np.empty((D, r), np.float32)
+    _check(lib.respin_factors_from_subspace(D, r, Q.ctypes.data_as(fp), R.ctypes.data_as(fp),
+                                            U.ctypes.data_as(fp), V.ctypes.data_as(fp)))
+    return U, V
+
+
+def respin_factors_from_transition(T, r: int, gap_tol: float = 1e-6):
+    """(U_r, V_r, sigma) = top-r factors of T - I for the plan (host fp32
+    T [D, D]); sigma holds s_1 .. s_(r+1). Raises RespinError
+    (RESPIN_ERR_UNSUPPORTED) when s_r - s_(r+1) <= gap_tol s_1."""
+    T = np.ascontiguousarray(T, dtype=np.float32)
+    D = T.shape[0]
+    if T.shape != (D, D):
+        raise ValueError("T must be square")
+    fp = ctypes.POINTER(ctypes.c_float)
+    U = np.empty((D, int(r)), np.float32)
+    V = np.empty((D, int(r)), np.float32)
+    sig = np.zeros(int(r) + 1, np.float64)
+    _check(lib.respin_factors_from_transition(D, int(r), T.ctypes.data_as(fp), float(gap_tol),
+                                              U.ctypes.data_as(fp), V.ctypes.data_as(fp),
+                                              sig.ctypes.data_as(ctypes.POINTER(ctypes.c_double))))
+    return U, V, sig
 
 
 def respin_device_status() -> int:

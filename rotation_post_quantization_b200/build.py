@@ -1,6 +1,7 @@
 """Build the CUDA library (librespin.so) in-tree for sm_100a with nvcc.
 
-Usage: python -m rotation_post_quantization_b200.build [--verbose]
+Usage: python rotation_post_quantization_b200/build.py [--verbose]
+(run as a script: the package itself loads the library at import)
 """
 from __future__ import annotations
 

@@ -20,6 +20,7 @@
 #include "ptx.cuh"
 #include "boundary_kernels.cuh"
 #include "boundary_rowtile.cuh"
+#include "factor_builder.h"
 #include "w4a4_gemm_kernels.cuh"
 #include "w4a4_gemm_skinny.cuh"
 
@@ -724,6 +725,37 @@ respin_status_t w4a4_gemm(const uint8_t* q_act, const float* scale_act, const ui
 respin_status_t w4a4_gemm_i32(const uint8_t* q_act, const uint8_t* q_w, int N, int K, int O,
                               int32_t* acc_out, void* stream) {
   return gemm_common(q_act, nullptr, q_w, nullptr, N, K, O, acc_out, stream, true);
+}
+
+respin_status_t respin_factors_from_subspace(int D, int r, const float* Q, const float* R_sub, float* U_r,
+                                            float* V_r) {
+  t_last_error.clear();
+  if (host::factors_from_subspace(D, r, Q, R_sub, U_r, V_r) != host::BuildResult::kOk)
+    return fail(RESPIN_ERR_INVALID_ARG, "need 0 < r <= D and non-NULL Q, R_sub, U_r, V_r");
+  return ok();
+}
+
+respin_status_t respin_factors_from_transition(int D, int r, const float* T, double gap_tol, float* U_r,
+                                               float* V_r, double* sigma) {
+  t_last_error.clear();
+  if (!(gap_tol >= 0.0)) return fail(RESPIN_ERR_INVALID_ARG, "gap_tol must be >= 0");
+  double s[129] = {0.0};
+  if (r > 128) return fail(RESPIN_ERR_INVALID_ARG, "r=%d: at most 128", r);
+  switch (host::factors_from_transition(D, r, T, gap_tol, U_r, V_r, s)) {
+    case host::BuildResult::kOk:
+      break;
+    case host::BuildResult::kBadArg:
+      return fail(RESPIN_ERR_INVALID_ARG, "need 0 < r < D and non-NULL T, U_r, V_r");
+    case host::BuildResult::kNoGap:
+      if (sigma != nullptr) std::memcpy(sigma, s, sizeof(double) * (r + 1));
+      return fail(RESPIN_ERR_UNSUPPORTED,
+                  "s_r - s_(r+1) = %.3e - %.3e is not above gap_tol * s_1 = %.3e: the top-%d truncation is not unique",
+                  s[r - 1], s[r], gap_tol * s[0], r);
+    default:
+      return fail(RESPIN_ERR_UNSUPPORTED, "the subspace iteration did not converge");
+  }
+  if (sigma != nullptr) std::memcpy(sigma, s, sizeof(double) * (r + 1));
+  return ok();
 }
 
 respin_status_t respin_device_status(int* code) {
