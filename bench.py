@@ -6,9 +6,12 @@ One step = the whole path on one batch of tokens: the fused boundary kernel
 §2.2 and §3-§4) followed by the tcgen05 W4A4 GEMM that consumes its codes.
 Workload: Llama-2-7B-shaped, D = 4096, 2048 tokens per GPU, r = 32 (rank-64
 skew deviation, norm 0.1, 8 outlier channels x50), GEMM 4096 -> 11008 with
-INT4 weights uniform in [-8, 7]. Synthetic, seeded inputs.
+INT4 weights uniform in [-8, 7]. Synthetic, seeded inputs. --workload
+llama2_7b_w3a3 runs the same step with 3-bit activation and weight codes
+(W3A3); the other --workload names print the remaining configurations.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME]
 
 Under torchrun each rank processes its own 2048 tokens (weak scaling, no
 data-path collective); the time is the max over ranks.

@@ -135,7 +135,8 @@ def respin_plan_destroy(plan: Plan) -> None:
 
 def respin_boundary_forward(plan: Plan, x, residual, h_out, q_packed, scale,
                             stream=None) -> None:
-    """h' = residual (I + U_r V_r^T) + x, then per-token INT4 codes and scales.
+    """h' = residual (I + U_r V_r^T) + x, then per-token INT4 codes and scales
+    (3-bit codes in the same nibbles for a plan made with RESPIN_ACT_INT3).
 
     x, residual, h_out: [N, D] CUDA tensors (bf16; h_out fp32 for a plan made
     with RESPIN_H_FP32_DEBUG; residual / h_out may be None); q_packed: uint8
