@@ -74,11 +74,13 @@ def test_ranks_hold_different_inputs():
     assert bench.rank_seed(0, 0) == 0
 
 
-def test_reference_arm_under_torchrun_two_ranks():
+@pytest.mark.parametrize("workload,bits", [("llama2_7b", 4), ("llama2_7b_w3a3", 3)])
+def test_reference_arm_under_torchrun_two_ranks(workload, bits):
     port = free_port()
     cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node=2",
            "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.join(ROOT, "bench.py"),
-           "--impl", "reference", "--gpus", "2", "--steps", "1", "--warmup", "0"]
+           "--impl", "reference", "--gpus", "2", "--steps", "1", "--warmup", "0",
+           "--workload", workload]
     env = dict(os.environ, OMP_NUM_THREADS="1")
     res = subprocess.run(cmd, capture_output=True, text=True, timeout=600, cwd=ROOT, env=env)
     assert res.returncode == 0, res.stderr[-2000:]
@@ -88,3 +90,4 @@ def test_reference_arm_under_torchrun_two_ranks():
     assert line["impl"] == "reference" and line["n_gpus"] == 2
     assert line["cpu_baseline"]["kind"] == "oracle"
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["value"] > 0
+    assert line["config"]["act_bits"] == bits and ("INT%d" % bits) in line["metric"]
