@@ -147,23 +147,23 @@ class ClockSampler(threading.Thread):
 # ---------------------------------------------------------------- oracle legs
 
 def oracle_sample_rate(fx, qw, sw, n_boundary: int, n_gemm: int, bits: int = 4):
-    """Time the CPU oracle (as it stands) on a bounded sample; tokens/s of
-    the whole path per token = 1 / (t_boundary/token + t_gemm/token)."""
+    """Time the C++ oracle (as it stands: plain single-threaded loops) on a
+    bounded sample; tokens/s of the whole path per token =
+    1 / (t_boundary/token + t_gemm/token)."""
     import numpy as np
-    from threadpoolctl import threadpool_limits
+    import torch
 
-    import oracle as O
-    with threadpool_limits(limits=1):
-        x = fx.x[:n_boundary].float().numpy()
-        res = fx.residual[:n_boundary].float().numpy()
-        U32, V32 = fx.U.astype(np.float32), fx.V.astype(np.float32)
-        t0 = time.perf_counter()
-        _, _, codes, scale = O.boundary_reference(x, res, U32, V32, 7 if bits == 4 else 3)
-        t1 = time.perf_counter()
-        qa = O.pack_int4(codes[:n_gemm])
-        acc = O.w4a4_acc(qa, qw)
-        O.w4a4_epilogue_bits(acc, scale[:n_gemm], sw)
-        t2 = time.perf_counter()
+    from oracle import native
+    native.lib()   # built before the clock starts
+    xb = fx.x[:n_boundary].view(torch.int16).numpy().view(np.uint16)
+    rb = fx.residual[:n_boundary].view(torch.int16).numpy().view(np.uint16)
+    U32, V32 = fx.U.astype(np.float32), fx.V.astype(np.float32)
+    t0 = time.perf_counter()
+    _, _, codes, scale = native.boundary_reference(xb, rb, U32, V32, 7 if bits == 4 else 3, want_h64=False)
+    t1 = time.perf_counter()
+    qa = native.pack(codes[:n_gemm])
+    native.w4a4_gemm(qa, scale[:n_gemm], qw, sw)
+    t2 = time.perf_counter()
     per_tok = (t1 - t0) / n_boundary + (t2 - t1) / n_gemm
     return 1.0 / per_tok, (t2 - t0)
 
@@ -183,12 +183,12 @@ def host_cpu() -> str:
 
 
 def cpu_baseline_block(fx, qw, sw, bits: int = 4):
-    rate, secs = oracle_sample_rate(fx, qw, sw, 2048, 160, bits)
+    rate, secs = oracle_sample_rate(fx, qw, sw, 2048, 400, bits)
     return {"value": rate, "unit": "tokens/s", "cores": 1, "kind": "oracle", "cpu": host_cpu(),
-            "sample": "boundary oracle (fp64 fix + binary32 INT%d quantizer) on all "
-                      "2048 tokens, W%dA%d GEMM oracle (exact int64 + binary32 "
-                      "epilogue) on 160 of the 2048 rows x 11008 channels; "
-                      "per-token times summed; %.1f s of CPU work, 1 thread"
+            "sample": "C++ oracle (plain loops, -O2, one thread): boundary (fp64 fix + "
+                      "binary32 INT%d quantizer) on all 2048 tokens, W%dA%d GEMM (exact "
+                      "int64 + binary32 epilogue) on 400 of the 2048 rows x 11008 "
+                      "channels; per-token times summed; %.1f s of CPU work"
                       % (bits, bits, bits, secs)}
 
 
@@ -213,7 +213,7 @@ def run_reference(args, rank: int):
         return
     bits = STEP_BITS.get(args.workload, 4)
     w, fx, qw, sw = workload_inputs(None, bits)
-    nb, ng = 64, 4
+    nb, ng = 256, 16
     for _ in range(max(0, args.warmup)):
         oracle_sample_rate(fx, qw, sw, nb, ng, bits)
     t = 0.0
@@ -234,8 +234,8 @@ def run_reference(args, rank: int):
         "config": config_block(w, args.gpus, bits),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1,
                          "kind": "oracle", "cpu": host_cpu(),
-                         "sample": "each step: boundary oracle on 64 tokens "
-                                   "+ GEMM oracle on 4 rows, 1 thread; "
+                         "sample": "each step: C++ oracle, boundary on 256 tokens "
+                                   "+ GEMM on 16 rows, 1 thread; "
                                    "%.1f s total" % t},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
