@@ -197,7 +197,8 @@ respin_status_t respin_factors_from_subspace(int D, int r, const float* Q,
  *   U_r,V_r : HOST fp32 [D, r] outputs (caller-owned).
  *   sigma   : HOST fp64 [r + 1] output s_1 .. s_(r+1), or NULL. Also written
  *             when the gap check refuses.
- * Host only; O(D^2 r) work per iteration. Errors: INVALID_ARG, UNSUPPORTED.
+ * Host only; O(D^2 r) work per iteration, 8 D^2 bytes of host memory for
+ * the float64 copy of T. Errors: INVALID_ARG, UNSUPPORTED, OOM.
  */
 respin_status_t respin_factors_from_transition(int D, int r, const float* T,
                                                double gap_tol, float* U_r,

@@ -12,6 +12,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <new>
 #include <set>
 #include <string>
 #include <vector>
@@ -741,7 +742,13 @@ respin_status_t respin_factors_from_transition(int D, int r, const float* T, dou
   if (!(gap_tol >= 0.0)) return fail(RESPIN_ERR_INVALID_ARG, "gap_tol must be >= 0");
   double s[129] = {0.0};
   if (r > 128) return fail(RESPIN_ERR_INVALID_ARG, "r=%d: at most 128", r);
-  switch (host::factors_from_transition(D, r, T, gap_tol, U_r, V_r, s)) {
+  host::BuildResult res;
+  try {   // float64 copies of T (D x D) and of the iteration blocks
+    res = host::factors_from_transition(D, r, T, gap_tol, U_r, V_r, s);
+  } catch (const std::bad_alloc&) {
+    return fail(RESPIN_ERR_OOM, "host memory for the %d x %d float64 transition", D, D);
+  }
+  switch (res) {
     case host::BuildResult::kOk:
       break;
     case host::BuildResult::kBadArg:
