@@ -196,3 +196,33 @@ def test_repeat_calls_deterministic():
     b = run_boundary(fx, f32=False)
     for k in a:
         assert np.array_equal(a[k], b[k])
+
+
+def test_rank_sweep_eckart_young_70b():
+    """Config-5 rank sweep on 256 tokens (D = 8192, Student-t, 16 outlier
+    channels x100, rank-128 Delta T): the fp32 h' of the rank-r fix against
+    the dense h = residual T + x (exact rank-128 factors, float64). Per token
+    the error stays within the Eckart-Young bound s_(r+1) |residual| plus the
+    bf16 rounding of the plan's factors (at most 1 % of s_1 |residual|) and
+    fp32 arithmetic, and its mean falls as r grows (it §2C, fr §2C: top-r
+    SVD; s_j = 2 |sin(theta_j / 2)|, each twice)."""
+    w = W.WORKLOADS["llama2_70b"]
+    D, k, nu, n = w.D, w.k, w.nu, 256
+    Q = W.orthonormal_basis(D, k, 0)
+    th = W.plane_angles(k, nu)
+    Uk, Vk = W.lowrank_factors(Q, th, k)
+    sig = np.repeat(2 * np.abs(np.sin(th / 2)), 2)
+    means = []
+    for r in w.extra["ranks"]:
+        fx = W.boundary_fixture(D, n, r, k=k, nu=nu, n_outlier=w.n_outlier,
+                                outlier_scale=w.outlier_scale, dist=w.dist)
+        got = run_boundary(fx, f32=True)
+        x = fx.x.float().numpy().astype(np.float64)
+        res = fx.residual.float().numpy().astype(np.float64)
+        hd = O.boundary_fp64(x, res, Uk, Vk)
+        e = np.linalg.norm(got["h"].astype(np.float64) - hd, axis=1)
+        rn = np.linalg.norm(res, axis=1)
+        bound = (sig[r] if r < k else 0.0) * rn + 0.01 * sig[0] * rn + 1e-5 * np.linalg.norm(hd, axis=1)
+        assert np.all(e <= bound), (r, float(np.max(e / bound)))
+        means.append(float(np.mean(e / rn)))
+    assert all(a > b for a, b in zip(means, means[1:])), means
