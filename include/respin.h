@@ -206,8 +206,20 @@ respin_status_t respin_factors_from_transition(int D, int r, const float* T,
 
 /* respin_device_status -- synchronizes the current device, then returns and
  * clears the device status word through *code (0 = no kernel gave up; else
- * the site that gave up). Returns DEVICE_CHECK if *code != 0. */
+ * the site of the first wait that gave up since the last clear). Returns
+ * DEVICE_CHECK if *code != 0. The outputs of a launch in which a wait gave up
+ * are invalid (the kernel skips its stores after the failure); the status
+ * word itself never changes what a later launch computes. */
 respin_status_t respin_device_status(int* code);
+
+/* respin_selftest_wait_limit -- failure-detection self test (for tests).
+ * Enqueues a one-thread kernel whose bounded mbarrier wait has nothing to
+ * wait for: after limit_us microseconds (1 .. 2,000,000) it gives up,
+ * records site 901 in the device status word (unless an earlier failure is
+ * recorded there) and returns. Nothing is copied or stored. The next
+ * respin_device_status() then reports DEVICE_CHECK with code 901 and clears
+ * the word. Errors: INVALID_ARG, CUDA. */
+respin_status_t respin_selftest_wait_limit(unsigned limit_us, void* stream);
 
 /* respin_last_error -- message of the last failed call on this thread (empty
  * string if none). The pointer stays valid until the next call on this

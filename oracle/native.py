@@ -42,9 +42,10 @@ def lib() -> ctypes.CDLL:
         L = ctypes.CDLL(LIB_PATH)
         vp, i32 = ctypes.c_void_p, ctypes.c_int
         L.oracle_boundary.argtypes = [i32, i32, i32, vp, vp, vp, vp, i32, vp, vp, vp, vp]
+        L.oracle_boundary_subspace.argtypes = [i32, i32, i32, vp, vp, vp, vp, i32, vp, vp, vp, vp]
         L.oracle_pack.argtypes = [i32, i32, vp, vp]
         L.oracle_w4a4.argtypes = [i32, i32, i32, vp, vp, vp, vp, vp, vp]
-        for f in (L.oracle_boundary, L.oracle_pack, L.oracle_w4a4):
+        for f in (L.oracle_boundary, L.oracle_boundary_subspace, L.oracle_pack, L.oracle_w4a4):
             f.restype = i32
         _lib = L
     return _lib
@@ -72,6 +73,26 @@ def boundary_reference(x_bits, res_bits, U32, V32, qmax: int = 7, want_h64: bool
                                _p(codes), _p(scale))
     if st != 0:
         raise ValueError("oracle_boundary: bad arguments")
+    return h64, hb, codes, scale
+
+
+def boundary_reference_subspace(x_bits, res_bits, Q32, R32, qmax: int = 7, want_h64: bool = True):
+    """As boundary_reference, for a plan in the stored subspace form: float32
+    basis Q [D, r] and rotation R_sub [r, r] (zh §2.2)."""
+    x = np.ascontiguousarray(x_bits, np.uint16)
+    N, D = x.shape
+    res = None if res_bits is None else np.ascontiguousarray(res_bits, np.uint16)
+    Q = np.ascontiguousarray(Q32, np.float32)
+    R = np.ascontiguousarray(R32, np.float32)
+    r = Q.shape[1] if Q.ndim == 2 else 0
+    h64 = np.empty((N, D), np.float64) if want_h64 else None
+    hb = np.empty((N, D), np.uint16)
+    codes = np.empty((N, D), np.int8)
+    scale = np.empty(N, np.float32)
+    st = lib().oracle_boundary_subspace(N, D, r, _p(x), _p(res), _p(Q), _p(R), int(qmax), _p(h64),
+                                        _p(hb), _p(codes), _p(scale))
+    if st != 0:
+        raise ValueError("oracle_boundary_subspace: bad arguments")
     return h64, hb, codes, scale
 
 

@@ -157,6 +157,23 @@ def boundary_fp64(x: np.ndarray, residual: np.ndarray | None,
     return h
 
 
+def boundary_subspace_fp64(x: np.ndarray, residual: np.ndarray | None,
+                           Q: np.ndarray, M: np.ndarray) -> np.ndarray:
+    """Row form of the zh §2.2 subspace residual rotation, float64 [N, D]:
+    y = residual Q (step 1, projection), z = y M^T (step 2, M = R_sub - I
+    inside the subspace), h' = residual + x + z Q^T (step 3, re-projection
+    and residual). A row h maps as h^T does in the column form."""
+    h = np.asarray(x, np.float64).copy()
+    if residual is not None:
+        res = np.asarray(residual, np.float64)
+        h += res
+        if Q.shape[1]:
+            y = res @ np.asarray(Q, np.float64)          # step 1
+            z = y @ np.asarray(M, np.float64).T          # step 2
+            h += z @ np.asarray(Q, np.float64).T         # step 3
+    return h
+
+
 def dense_boundary_fp64(x: np.ndarray, residual: np.ndarray,
                         P: np.ndarray) -> np.ndarray:
     """h' = residual P + x with the dense D x D operator, float64."""
@@ -321,6 +338,26 @@ def boundary_reference(x, residual, U32, V32, qmax: int = 7):
     """
     Uq, Vq = plan_factors(U32, V32)
     h64 = boundary_fp64(x, residual, Uq, Vq)
+    hb = bf16_bits(h64)
+    codes, scale = quantize_per_token(bf16_bits_to_f32(hb), qmax)
+    return h64, hb, codes, scale
+
+
+def subspace_plan_factors(Q, R_sub):
+    """The stored subspace form as the plan holds it: the float32 basis Q
+    rounded to bfloat16, and M = R_sub - I from the float32 rotation, the
+    difference taken exactly and rounded once to binary32; both returned as
+    float64 values."""
+    R = np.asarray(R_sub, np.float32).astype(np.float64)
+    M = (R - np.eye(R.shape[0])).astype(np.float32).astype(np.float64)
+    return round_to_bf16(np.asarray(Q, np.float32)), M
+
+
+def boundary_reference_subspace(x, residual, Q32, R32, qmax: int = 7):
+    """boundary_reference for a plan made from the stored subspace form
+    (float32 Q [D, r] and R_sub [r, r], zh §2.2)."""
+    Qq, M = subspace_plan_factors(Q32, R32)
+    h64 = boundary_subspace_fp64(x, residual, Qq, M)
     hb = bf16_bits(h64)
     codes, scale = quantize_per_token(bf16_bits_to_f32(hb), qmax)
     return h64, hb, codes, scale

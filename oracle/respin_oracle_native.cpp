@@ -8,6 +8,12 @@
 //
 //   factors    : the plan's bfloat16 copies of U_r, V_r (round to nearest even)
 //   boundary   : h = (residual + x) + (residual U) V^T     in float64, plain loops
+//   subspace   : the stored form of zh §2.2 (basis Q, rotation R_sub): the plan
+//                holds bfloat16(Q) and M = float(R_sub - I) (difference exact,
+//                one rounding to binary32); per token, in float64 and in the
+//                page's step order: y = residual Q (projection), z = y M^T
+//                (transform inside the subspace), h = residual + x + z Q^T
+//                (re-projection and residual)
 //   h'         : bfloat16(h), one rounding to nearest even
 //   quantizer  : binary32 on g = float(h'): amax = max|g|; amax < 2^-125 gives
 //                scale 0 and zero codes; else inv = qmax / amax,
@@ -56,6 +62,35 @@ float bf16_to_float(uint16_t b) {
   return f;
 }
 
+// Quantizer of one token (binary32 on the bfloat16-rounded h'): fills hbits,
+// h64 (if given), codes and *scale.
+void quantize_token(const double* h, int D, int qmax, double* h64, uint16_t* hbits, int8_t* c, float* scale,
+                    std::vector<float>& g) {
+  const float qm = static_cast<float>(qmax);
+  float amax = 0.0f;
+  for (int d = 0; d < D; ++d) {
+    const uint16_t b = bf16_bits_of(h[d]);
+    hbits[d] = b;
+    if (h64 != nullptr) h64[d] = h[d];
+    g[d] = bf16_to_float(b);
+    amax = std::fmax(amax, std::fabs(g[d]));
+  }
+  if (!(amax >= kZeroTokenAmax)) {
+    *scale = 0.0f;
+    for (int d = 0; d < D; ++d) c[d] = 0;
+    return;
+  }
+  const float inv = qm / amax;
+  for (int d = 0; d < D; ++d) {
+    const float t = g[d] * inv;
+    float q = std::nearbyint(t);
+    if (q > qm) q = qm;
+    if (q < -qm - 1.0f) q = -qm - 1.0f;
+    c[d] = static_cast<int8_t>(q);
+  }
+  *scale = amax / qm;
+}
+
 int nibble(const uint8_t* row, int k) {
   const int v = (k & 1) ? (row[k >> 1] >> 4) : (row[k >> 1] & 0xF);
   return v >= 8 ? v - 16 : v;
@@ -83,7 +118,6 @@ int oracle_boundary(int N, int D, int r, const uint16_t* x, const uint16_t* res,
   }
   std::vector<double> h(D), y(r);
   std::vector<float> g(D);
-  const float qm = static_cast<float>(qmax);
   for (int n = 0; n < N; ++n) {
     const uint16_t* xr = x + static_cast<size_t>(n) * D;
     for (int d = 0; d < D; ++d) h[d] = bf16_to_float(xr[d]);
@@ -101,29 +135,55 @@ int oracle_boundary(int N, int D, int r, const uint16_t* x, const uint16_t* res,
         h[d] += c;
       }
     }
-    float amax = 0.0f;
-    for (int d = 0; d < D; ++d) {
-      const uint16_t b = bf16_bits_of(h[d]);
-      hbits[static_cast<size_t>(n) * D + d] = b;
-      if (h64 != nullptr) h64[static_cast<size_t>(n) * D + d] = h[d];
-      g[d] = bf16_to_float(b);
-      amax = std::fmax(amax, std::fabs(g[d]));
+    const size_t o = static_cast<size_t>(n) * D;
+    quantize_token(h.data(), D, qmax, h64 != nullptr ? h64 + o : nullptr, hbits + o, codes + o, scale + n, g);
+  }
+  return 0;
+}
+
+// The same call with the plan in the stored subspace form: Q float [D][r],
+// R_sub float [r][r] (row-major). Plan values: bfloat16(Q) and
+// M = float(R_sub - I). Returns 0, or -1 for a bad argument.
+int oracle_boundary_subspace(int N, int D, int r, const uint16_t* x, const uint16_t* res, const float* Q,
+                             const float* R_sub, int qmax, double* h64, uint16_t* hbits, int8_t* codes,
+                             float* scale) {
+  if (N < 0 || D <= 0 || r < 0 || x == nullptr || hbits == nullptr || codes == nullptr || scale == nullptr ||
+      (qmax != 7 && qmax != 3) || (res != nullptr && r > 0 && (Q == nullptr || R_sub == nullptr)))
+    return -1;
+  std::fesetround(FE_TONEAREST);
+  std::vector<double> Qq(static_cast<size_t>(D) * r), M(static_cast<size_t>(r) * r);
+  for (size_t i = 0; i < Qq.size(); ++i) Qq[i] = bf16_to_float(bf16_bits_of(Q[i]));
+  for (int i = 0; i < r; ++i)
+    for (int j = 0; j < r; ++j) {
+      const double d = static_cast<double>(R_sub[static_cast<size_t>(i) * r + j]) - (i == j ? 1.0 : 0.0);
+      M[static_cast<size_t>(i) * r + j] = static_cast<double>(static_cast<float>(d));
     }
-    int8_t* c = codes + static_cast<size_t>(n) * D;
-    if (!(amax >= kZeroTokenAmax)) {
-      scale[n] = 0.0f;
-      for (int d = 0; d < D; ++d) c[d] = 0;
-      continue;
+  std::vector<double> h(D), y(r), z(r);
+  std::vector<float> g(D);
+  for (int n = 0; n < N; ++n) {
+    const uint16_t* xr = x + static_cast<size_t>(n) * D;
+    for (int d = 0; d < D; ++d) h[d] = bf16_to_float(xr[d]);
+    if (res != nullptr) {
+      const uint16_t* rr = res + static_cast<size_t>(n) * D;
+      for (int d = 0; d < D; ++d) h[d] += bf16_to_float(rr[d]);        // residual + x
+      for (int j = 0; j < r; ++j) y[j] = 0.0;
+      for (int d = 0; d < D; ++d) {                                       // step 1: y = residual Q
+        const double v = bf16_to_float(rr[d]);
+        for (int j = 0; j < r; ++j) y[j] += v * Qq[static_cast<size_t>(d) * r + j];
+      }
+      for (int i = 0; i < r; ++i) {                                       // step 2: z = y M^T
+        double a = 0.0;
+        for (int j = 0; j < r; ++j) a += y[j] * M[static_cast<size_t>(i) * r + j];
+        z[i] = a;
+      }
+      for (int d = 0; d < D; ++d) {                                       // step 3: + z Q^T
+        double c = 0.0;
+        for (int i = 0; i < r; ++i) c += z[i] * Qq[static_cast<size_t>(d) * r + i];
+        h[d] += c;
+      }
     }
-    const float inv = qm / amax;
-    for (int d = 0; d < D; ++d) {
-      const float t = g[d] * inv;
-      float q = std::nearbyint(t);
-      if (q > qm) q = qm;
-      if (q < -qm - 1.0f) q = -qm - 1.0f;
-      c[d] = static_cast<int8_t>(q);
-    }
-    scale[n] = amax / qm;
+    const size_t o = static_cast<size_t>(n) * D;
+    quantize_token(h.data(), D, qmax, h64 != nullptr ? h64 + o : nullptr, hbits + o, codes + o, scale + n, g);
   }
   return 0;
 }

@@ -29,7 +29,8 @@ RESPIN_ACT_INT3 = 2
 EXPORTED = ("respin_plan_create", "respin_plan_destroy",
             "respin_boundary_forward", "w4a4_gemm", "w4a4_gemm_i32",
             "respin_factors_from_subspace", "respin_factors_from_transition",
-            "respin_device_status", "respin_last_error", "respin_version")
+            "respin_device_status", "respin_selftest_wait_limit",
+            "respin_last_error", "respin_version")
 
 
 class RespinError(RuntimeError):
@@ -58,6 +59,7 @@ def _load() -> ctypes.CDLL:
     lib.respin_factors_from_subspace.argtypes = [i32, i32, fp, fp, fp, fp]
     lib.respin_factors_from_transition.argtypes = [i32, i32, fp, ctypes.c_double, fp, fp, dp]
     lib.respin_device_status.argtypes = [ctypes.POINTER(ctypes.c_int)]
+    lib.respin_selftest_wait_limit.argtypes = [u32, vp]
     for name in EXPORTED[:-2]:
         getattr(lib, name).restype = ctypes.c_int
     lib.respin_last_error.restype = ctypes.c_char_p
@@ -202,6 +204,12 @@ def respin_factors_from_transition(T, r: int, gap_tol: float = 1e-6):
                                               U.ctypes.data_as(fp), V.ctypes.data_as(fp),
                                               sig.ctypes.data_as(ctypes.POINTER(ctypes.c_double))))
     return U, V, sig
+
+
+def respin_selftest_wait_limit(limit_us: int, stream=None) -> None:
+    """Enqueue the failure-detection self test: a bounded wait that nothing
+    completes gives up after limit_us microseconds and records site 901."""
+    _check(lib.respin_selftest_wait_limit(int(limit_us), _stream(stream)))
 
 
 def respin_device_status() -> int:

@@ -125,7 +125,7 @@ __device__ __forceinline__ void load_n8(uint32_t (&w)[MT][2][2], const uint8_t* 
 template <bool F32OUT>
 __device__ __forceinline__ void finish_n8(const float (&acc)[4], const uint32_t (&w)[2][2], uint8_t* xs_ptr,
                                           uint32_t pitch, int rowA, int colc, float (&rmax)[2],
-                                          void* h_out, int row0, int N, int D, int col0) {
+                                          void* h_out, int row0, int N, int D, int col0, bool ok) {
 #pragma unroll
   for (int hh = 0; hh < 2; ++hh) {
     const int row = rowA + 8 * hh;
@@ -137,7 +137,7 @@ __device__ __forceinline__ void finish_n8(const float (&acc)[4], const uint32_t 
     *reinterpret_cast<uint32_t*>(xs_ptr + off) = hb;
     rmax[hh] = fmaxf(rmax[hh], fmaxf(fabsf(bf16_lo_f32(hb)), fabsf(bf16_hi_f32(hb))));
     if constexpr (F32OUT) {
-      if (h_out != nullptr && row0 + row < N) {
+      if (ok && h_out != nullptr && row0 + row < N) {
         float* hf = static_cast<float*>(h_out) + static_cast<size_t>(row0 + row) * D + col0 + colc;
         *reinterpret_cast<float2*>(hf) = make_float2(h0, h1);
       }
@@ -146,10 +146,11 @@ __device__ __forceinline__ void finish_n8(const float (&acc)[4], const uint32_t 
 }
 
 // Row amax: per-thread row maxima -> warp maxima in `wamax` [8][T] -> after a
-// CTA barrier the T row maxima of this CTA's slice in `amaxbuf`.
+// CTA barrier the T row maxima of this CTA's slice in `amaxbuf`. Returns `ok`
+// ANDed over the CTA (taken at that barrier).
 template <int MT, int T>
-__device__ __forceinline__ void publish_amax(float (&rmax)[MT][2], float* wamax, float* amaxbuf,
-                                             int warp, int lane, int tid) {
+__device__ __forceinline__ bool publish_amax(float (&rmax)[MT][2], float* wamax, float* amaxbuf,
+                                             int warp, int lane, int tid, bool ok) {
   const int g = lane >> 2, q4 = lane & 3;
 #pragma unroll
   for (int mt = 0; mt < MT; ++mt)
@@ -160,13 +161,14 @@ __device__ __forceinline__ void publish_amax(float (&rmax)[MT][2], float* wamax,
       m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
       if (q4 == 0) wamax[warp * T + mt * 16 + g + 8 * hh] = m;
     }
-  __syncthreads();
+  ok = __syncthreads_and(ok) != 0;
   if (tid < T) {
     float m = 0.f;
 #pragma unroll
     for (int w = 0; w < 8; ++w) m = fmaxf(m, wamax[w * T + tid]);
     amaxbuf[tid] = m;
   }
+  return ok;
 }
 
 // After the amax cluster barrier: gather every CTA's row maxima in parallel
@@ -174,7 +176,7 @@ __device__ __forceinline__ void publish_amax(float (&rmax)[MT][2], float* wamax,
 template <int T>
 __device__ __forceinline__ void gather_amax(uint32_t amaxbuf_addr, float* am2, float* rowinv,
                                             float* scale_out, uint32_t csize, uint32_t crank,
-                                            int row0, int N, int tid, float qmax) {
+                                            int row0, int N, int tid, float qmax, bool ok) {
   for (int i = tid; i < static_cast<int>(csize) * T; i += kBoundaryThreads) {
     const uint32_t c = static_cast<uint32_t>(i / T);
     am2[i] = ld_dsmem_f32(map_to_rank(amaxbuf_addr + 4u * (i % T), c));
@@ -186,7 +188,7 @@ __device__ __forceinline__ void gather_amax(uint32_t amaxbuf_addr, float* am2, f
     float inv, sc;
     inv_and_scale(m, qmax, inv, sc);
     rowinv[tid] = inv;
-    if (crank == 0 && row0 + tid < N) scale_out[row0 + tid] = sc;
+    if (ok && crank == 0 && row0 + tid < N) scale_out[row0 + tid] = sc;
   }
   __syncthreads();
 }
@@ -195,9 +197,9 @@ __device__ __forceinline__ void gather_amax(uint32_t amaxbuf_addr, float* am2, f
 template <bool F32OUT>
 __device__ __forceinline__ void store_tile(const uint8_t* xs_ptr, uint32_t pitch, const float* rowinv,
                                            int T, int Dc, int row0, int N, int D, int col0,
-                                           void* h_out, uint8_t* q_out, int tid) {
+                                           void* h_out, uint8_t* q_out, int tid, bool ok) {
   const int vpr = Dc / 8;
-  for (int i = tid; i < T * vpr; i += kBoundaryThreads) {
+  for (int i = tid; ok && i < T * vpr; i += kBoundaryThreads) {
     const int row = i / vpr, v = i % vpr;
     if (row0 + row >= N) continue;
     const uint4 hv = *reinterpret_cast<const uint4*>(xs_ptr + row * pitch + v * 16);
@@ -292,11 +294,18 @@ boundary_cluster_rf_kernel(const bf16* __restrict__ x, const bf16* __restrict__ 
   }
   __syncthreads();
 
+  // ok: false once a wait of this CTA gave up (CTA-uniform at the CTA
+  // barriers). From then on no copy is issued and nothing is stored; waits
+  // still run for copies already issued, so none is in flight at exit.
+  bool ok = true;
+  int issued[2] = {0, 0};   // loop iterations whose residual / x copies were issued
   // Warp 0: bulk-copy the residual (which = 0) or x (which = 1) rows of loop
   // iteration `it` into stage it % S.
   auto issue = [&](int it, int which) {
     const int tile = static_cast<int>(cid) + it * static_cast<int>(ncl);
-    if (warp != 0 || tile >= ntiles) return;
+    if (!ok || tile >= ntiles) return;
+    issued[which] = it + 1;
+    if (warp != 0) return;
     const int s = it % S;
     const int row0 = tile * T;
     const int rows = min(T, N - row0);
@@ -352,7 +361,7 @@ boundary_cluster_rf_kernel(const bf16* __restrict__ x, const bf16* __restrict__ 
     uint8_t* xs_ptr = smem + s * C::kStage + T * pitch;
 
     // ---- phase 1: this CTA's partial y = residual[:, slice] U_slice
-    mbar_wait(bars + 8 * s, par, kSiteBoundaryLoad);
+    if (it < issued[0]) ok = mbar_wait(bars + 8 * s, par, kSiteBoundaryLoad) && ok;
     {
       float acc[C::NPW][4];
 #pragma unroll
@@ -374,7 +383,7 @@ boundary_cluster_rf_kernel(const bf16* __restrict__ x, const bf16* __restrict__ 
         *reinterpret_cast<float2*>(&pw[(row + 8) * RP + col]) = make_float2(acc[p][2], acc[p][3]);
       }
     }
-    __syncthreads();
+    ok = __syncthreads_and(ok) != 0;
     if (tid < T * R / 4) {
       const int e = 4 * tid, row = e / R, col = e % R;
       float4 sum = *reinterpret_cast<const float4*>(&part[row * RP + col]);
@@ -399,7 +408,7 @@ boundary_cluster_rf_kernel(const bf16* __restrict__ x, const bf16* __restrict__ 
     __syncthreads();
 
     // ---- phase 2: h = (res + x) + y V_slice^T, bf16 round, row amax
-    mbar_wait(bars + 8 * (S + s), par, kSiteBoundaryLoad);
+    if (it < issued[1]) ok = mbar_wait(bars + 8 * (S + s), par, kSiteBoundaryLoad) && ok;
     {
       uint32_t ahi[C::MT][C::KS2][4], alo[C::MT][C::KS2][4];
 #pragma unroll
@@ -460,7 +469,7 @@ boundary_cluster_rf_kernel(const bf16* __restrict__ x, const bf16* __restrict__ 
                               __halves2bfloat162(__hmax(__low2bfloat16(mA), __high2bfloat16(mA)),
                                                  __hmax(__low2bfloat16(mB), __high2bfloat16(mB))));
           if constexpr (F32OUT) {
-            if (h_out != nullptr) {
+            if (h_out != nullptr && ok) {
               float* hf = static_cast<float*>(h_out) + col0 + d0 + 2 * q4;
               if (row0 + rowA < N)
                 *reinterpret_cast<float2*>(hf + static_cast<size_t>(row0 + rowA) * D) = make_float2(acc[0], acc[1]);
@@ -483,7 +492,7 @@ boundary_cluster_rf_kernel(const bf16* __restrict__ x, const bf16* __restrict__ 
           wamax[warp * T + mt * 16 + g + 8] = mB;
         }
       }
-      __syncthreads();
+      ok = __syncthreads_and(ok) != 0;
       if (tid < T) {
         float m = 0.f;
 #pragma unroll
@@ -505,7 +514,7 @@ boundary_cluster_rf_kernel(const bf16* __restrict__ x, const bf16* __restrict__ 
       float inv, sc;
       inv_and_scale(m, qmax, inv, sc);
       rowinv[tid] = inv;
-      if (crank == 0 && row0 + tid < N) scale_out[row0 + tid] = sc;
+      if (ok && crank == 0 && row0 + tid < N) scale_out[row0 + tid] = sc;
     }
     __syncthreads();
 
@@ -515,7 +524,7 @@ boundary_cluster_rf_kernel(const bf16* __restrict__ x, const bf16* __restrict__ 
 #pragma unroll 4
       for (int i = tid; i < T * vpr; i += kRfThreads) {
         const int row = i / vpr, v = i % vpr;
-        if (row0 + row >= N) continue;
+        if (!ok || row0 + row >= N) continue;
         const uint4 hv = *reinterpret_cast<const uint4*>(xs_ptr + row * pitch + v * 16);
         const size_t gi = static_cast<size_t>(row0 + row) * D + col0 + v * 8;
         if constexpr (!F32OUT) {
@@ -616,9 +625,16 @@ boundary_cluster_smem_kernel(const bf16* __restrict__ x, const bf16* __restrict_
   }
   __syncthreads();
 
+  // ok: false once a wait of this CTA gave up (CTA-uniform at the CTA
+  // barriers). From then on no copy is issued and nothing is stored; waits
+  // still run for copies already issued, so none is in flight at exit.
+  bool ok = true;
+  int issued = 0;   // loop iterations whose copies were issued
   auto issue = [&](int it) {
     const int tile = static_cast<int>(cid) + it * static_cast<int>(ncl);
-    if (tile >= ntiles || warp != 0) return;
+    if (!ok || tile >= ntiles) return;
+    issued = it + 1;
+    if (warp != 0) return;
     const int s = it & 1;
     const uint32_t st = sbase + L.stage0 + s * L.stage_bytes;
     stage_tile(x, res, tile * T, N, D, col0, Dc, T, st, st + T * pitch, pitch, bars + 16 * s,
@@ -663,7 +679,7 @@ boundary_cluster_smem_kernel(const bf16* __restrict__ x, const bf16* __restrict_
     uint8_t* xs_ptr = smem + L.stage0 + s * L.stage_bytes + T * pitch;
 
     // ---- phase 1: partial y = residual_tile[:, slice] * U_slice (tensor cores)
-    mbar_wait(bars + 16 * s, par, kSiteBoundaryLoad);
+    if (it < issued) ok = mbar_wait(bars + 16 * s, par, kSiteBoundaryLoad) && ok;
     {
       const int wm = warp % C::MT;
       const int wn = (warp / C::MT) % C::WN;
@@ -697,7 +713,7 @@ boundary_cluster_smem_kernel(const bf16* __restrict__ x, const bf16* __restrict_
         *reinterpret_cast<float2*>(&pw[(row + 8) * RP + col]) = make_float2(acc[j][2], acc[j][3]);
       }
     }
-    __syncthreads();
+    ok = __syncthreads_and(ok) != 0;
     for (int e = tid * 4; e < T * R; e += kBoundaryThreads * 4) {
       const int row = e / R, col = e % R;
       float4 sum = *reinterpret_cast<const float4*>(&part[row * RP + col]);
@@ -719,7 +735,7 @@ boundary_cluster_smem_kernel(const bf16* __restrict__ x, const bf16* __restrict_
     __syncthreads();
 
     // ---- phase 2: h = (res + x) + y V_slice^T, bf16 round, row amax
-    mbar_wait(bars + 16 * s + 8, par, kSiteBoundaryLoad);
+    if (it < issued) ok = mbar_wait(bars + 16 * s + 8, par, kSiteBoundaryLoad) && ok;
     {
       uint32_t ahi[C::MT][C::KS2][4], alo[C::MT][C::KS2][4];
 #pragma unroll
@@ -779,7 +795,7 @@ boundary_cluster_smem_kernel(const bf16* __restrict__ x, const bf16* __restrict_
 #pragma unroll
         for (int mt = 0; mt < C::MT; ++mt)
           finish_n8<F32OUT>(acc[mt], wcur[mt], xs_ptr, pitch, mt * 16 + g, d0 + 2 * q4, rmax[mt], h_out, row0,
-                            N, D, col0);
+                            N, D, col0, ok);
 #pragma unroll
         for (int mt = 0; mt < C::MT; ++mt)
 #pragma unroll
@@ -788,13 +804,13 @@ boundary_cluster_smem_kernel(const bf16* __restrict__ x, const bf16* __restrict_
             wcur[mt][hh][1] = wnext[mt][hh][1];
           }
       }
-      publish_amax<C::MT, T>(rmax, wamax, amaxbuf, warp, lane, tid);
+      ok = publish_amax<C::MT, T>(rmax, wamax, amaxbuf, warp, lane, tid, ok);
     }
 
     // ---- amax over the cluster, then codes
     cluster_sync();
-    gather_amax<T>(sbase + L.amaxbuf, am2, rowinv, scale_out, csize, crank, row0, N, tid, qmax);
-    store_tile<F32OUT>(xs_ptr, pitch, rowinv, T, Dc, row0, N, D, col0, h_out, q_out, tid);
+    gather_amax<T>(sbase + L.amaxbuf, am2, rowinv, scale_out, csize, crank, row0, N, tid, qmax, ok);
+    store_tile<F32OUT>(xs_ptr, pitch, rowinv, T, Dc, row0, N, D, col0, h_out, q_out, tid, ok);
     fence_proxy_async_smem();
     __syncthreads();
     issue(it + 2);

@@ -184,6 +184,12 @@ boundary_rowtile_kernel(const __grid_constant__ CUtensorMap tmR, const __grid_co
                 xbar0 + 8 * slot);
   };
   if (lane < XS) issue_x(lane);
+  // ok: false once a wait gave up (warp-uniform after each wait, CTA-uniform
+  // at the CTA barriers). From then on no copy is issued and nothing is
+  // stored; waits still run for copies already issued (uses u < x_issued of
+  // the x stream, tiles with res_issued), so none is in flight at exit.
+  int x_issued = XS;
+  bool res_issued = false;
 
   auto load_u = [&](uint4 (&dst)[C::UB], int j) {
     const uint4* src = Ut + static_cast<size_t>(warp * NB + j) * C::UB * 32 + lane;
@@ -202,7 +208,8 @@ boundary_rowtile_kernel(const __grid_constant__ CUtensorMap tmR, const __grid_co
     const int row0 = tile * kRtT;
     // ---- residual tile: lane j < NB loads block warp * NB + j (after its
     // own h' store of the previous tile has finished reading the block)
-    if (lane < NB) {
+    res_issued = ok;
+    if (ok && lane < NB) {
       const int b = warp * NB + lane;
       mbar_arrive_expect_tx(res_bar, kRtBlockBytes);
       tma_load_2d(tileA + b * kRtBlockBytes, &tmR, b * 64, row0, res_bar);
@@ -216,7 +223,7 @@ boundary_rowtile_kernel(const __grid_constant__ CUtensorMap tmR, const __grid_co
     float acc1[C::NT][4];
 #pragma unroll
     for (int p = 0; p < C::NT; ++p) acc1[p][0] = acc1[p][1] = acc1[p][2] = acc1[p][3] = 0.f;
-    if (ok) ok = mbar_wait(res_bar, it & 1, kSiteBoundaryLoad);
+    if (res_issued) ok = mbar_wait(res_bar, it & 1, kSiteBoundaryLoad) && ok;
     ok = __all_sync(0xffffffffu, ok);
 #pragma unroll
     for (int j = 0; j < NB; ++j) {
@@ -247,7 +254,7 @@ boundary_rowtile_kernel(const __grid_constant__ CUtensorMap tmR, const __grid_co
         *reinterpret_cast<float2*>(yp + (g + 8) * C::YP + 8 * p + 2 * q4) = make_float2(acc1[p][2], acc1[p][3]);
       }
     }
-    __syncthreads();
+    ok = __syncthreads_and(ok) != 0;
     if (tid < kRtT * R / 2) {
       const int row = tid / (R / 2), c2 = 2 * (tid % (R / 2));
       float2 s = make_float2(0.f, 0.f);
@@ -291,7 +298,8 @@ boundary_rowtile_kernel(const __grid_constant__ CUtensorMap tmR, const __grid_co
       if (j + RING - 1 < NB) load_v(vb[(j + RING - 1) % RING], j + RING - 1);
       const int u = it * NB + j;
       const int slot = u % XS;
-      if (ok) ok = mbar_wait(xbar0 + 8 * slot, (u / XS) & 1, kSiteBoundaryLoad);
+      if (u < x_issued) ok = mbar_wait(xbar0 + 8 * slot, (u / XS) & 1, kSiteBoundaryLoad) && ok;
+      ok = __all_sync(0xffffffffu, ok);
       uint8_t* blk = smem + (warp * NB + j) * kRtBlockBytes;
       const uint8_t* xblk = smem + C::x_ring(D) + (warp * XS + slot) * kRtBlockBytes;
       const int colb = (warp * NB + j) * 64;
@@ -341,7 +349,7 @@ boundary_rowtile_kernel(const __grid_constant__ CUtensorMap tmR, const __grid_co
             amax2[hh] = absmax_bf16x2(amax2[hh], hb);
             if constexpr (F32OUT) {
               const int row = g + 8 * hh;
-              if (h_out != nullptr && row0 + row < N)
+              if (ok && h_out != nullptr && row0 + row < N)
                 *reinterpret_cast<float2*>(static_cast<float*>(h_out) + static_cast<size_t>(row0 + row) * D +
                                            colb + 16 * q4 + 2 * t) = h;
             }
@@ -355,7 +363,10 @@ boundary_rowtile_kernel(const __grid_constant__ CUtensorMap tmR, const __grid_co
       // the slot's bytes were read (generic proxy) before its next tensor copy
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == slot) issue_x(u + XS);
+      if (ok) {
+        if (lane == slot) issue_x(u + XS);
+        x_issued = u + XS + 1;
+      }
     }
     float rmax[2];
 #pragma unroll
@@ -369,7 +380,7 @@ boundary_rowtile_kernel(const __grid_constant__ CUtensorMap tmR, const __grid_co
       m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
       if (q4 == 0) wamax[warp * kRtT + g + 8 * hh] = m;
     }
-    __syncthreads();
+    ok = __syncthreads_and(ok) != 0;
     if (tid < kRtT) {
       float m = 0.f;
 #pragma unroll
@@ -377,7 +388,7 @@ boundary_rowtile_kernel(const __grid_constant__ CUtensorMap tmR, const __grid_co
       float inv, sc;
       inv_and_scale(m, qmax, inv, sc);
       rowinv[tid] = inv;
-      if (row0 + tid < N) scale_out[row0 + tid] = sc;
+      if (ok && row0 + tid < N) scale_out[row0 + tid] = sc;
     }
     __syncthreads();
 

@@ -9,8 +9,11 @@
 namespace respin {
 
 // Device status word: 0 = fine, otherwise the site of the first bounded wait
-// that gave up. Read and cleared by respin_device_status(). The library is
-// compiled as a single translation unit, so this header is included once.
+// that gave up. Sticky across launches until respin_device_status() reads and
+// clears it; a later launch does not look at it (each wait gives up only on
+// its own time limit), so a stale code never cuts another launch short. The
+// library is compiled as a single translation unit, so this header is
+// included once.
 __device__ int g_status = 0;
 
 enum StatusSite : int {
@@ -20,6 +23,9 @@ enum StatusSite : int {
   kSiteGemmAccum = 203,      // GEMM epilogue / MMA: waiting for an accumulator buffer
   kSiteGemmPackedFull = 204, // GEMM producer: waiting for a packed K block (TMA)
   kSiteGemmPackedEmpty = 205,// GEMM TMA warp: waiting for a free packed stage
+  kSitePairPeer = 301,       // pair boundary kernel: waiting for the peer CTA's partials
+  kSitePairLoad = 302,       // pair boundary kernel: waiting for a staged block or the basis
+  kSiteSelfTest = 901,       // respin_selftest_wait_limit: a wait that nothing completes
 };
 
 // Upper bound on any single wait inside a kernel (nanoseconds of globaltimer).
@@ -33,10 +39,6 @@ __device__ __forceinline__ uint64_t globaltimer() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
-}
-
-__device__ __forceinline__ bool status_failed() {
-  return *reinterpret_cast<volatile int*>(&g_status) != 0;
 }
 
 __device__ __forceinline__ void record_status(int site) {
@@ -81,15 +83,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Wait for the phase with the given parity to complete. Gives up (returns
-// false and records `site`) after kWaitLimitNs, or at once if another wait in
-// this launch already gave up.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int site) {
+// false and records `site`) after `limit_ns` of %globaltimer. A caller that
+// gets false must treat what the phase guarded as invalid: skip its stores,
+// issue no further copies into that buffer, and before exiting wait (again
+// bounded) for any copy it issued and has not waited for.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int site,
+                                          uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (status_failed()) return false;
-    if (globaltimer() - t0 > kWaitLimitNs) {
+    if (globaltimer() - t0 > limit_ns) {
       record_status(site);
       return false;
     }
@@ -110,13 +114,13 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t par
   return ok != 0;
 }
 
-__device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity, int site) {
+__device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity, int site,
+                                                  uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait_cluster(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   while (true) {
     if (mbar_try_wait_cluster(bar, parity)) return true;
-    if (status_failed()) return false;
-    if (globaltimer() - t0 > kWaitLimitNs) {
+    if (globaltimer() - t0 > limit_ns) {
       record_status(site);
       return false;
     }

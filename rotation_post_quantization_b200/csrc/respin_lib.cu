@@ -765,6 +765,35 @@ respin_status_t respin_factors_from_transition(int D, int r, const float* T, dou
   return ok();
 }
 
+}  // extern "C"
+
+namespace {
+
+// One thread waits on an mbarrier that nothing arrives on, with the given
+// limit: the wait gives up and records kSiteSelfTest. Nothing is copied, so
+// nothing is in flight when the kernel returns.
+__global__ void selftest_wait_kernel(uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  const uint32_t b = smem_u32(&bar);
+  mbar_init(b, 1);
+  fence_mbarrier_init();
+  mbar_wait(b, 0, kSiteSelfTest, limit_ns);
+}
+
+}  // namespace
+
+extern "C" {
+
+respin_status_t respin_selftest_wait_limit(unsigned limit_us, void* stream) {
+  t_last_error.clear();
+  if (limit_us == 0 || limit_us > 2000000u)
+    return fail(RESPIN_ERR_INVALID_ARG, "limit_us=%u: need 1 <= limit_us <= 2000000", limit_us);
+  selftest_wait_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(static_cast<uint64_t>(limit_us) * 1000u);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "selftest_wait_kernel launch");
+  return ok();
+}
+
 respin_status_t respin_device_status(int* code) {
   t_last_error.clear();
   if (code == nullptr) return fail(RESPIN_ERR_INVALID_ARG, "code is NULL");

@@ -147,3 +147,9 @@ def test_last_error_cleared_on_success():
 
 def test_device_status_null():
     assert rq.lib.respin_device_status(None) == rq.RESPIN_ERR_INVALID_ARG
+
+
+def test_selftest_limit_validation():
+    assert rq.lib.respin_selftest_wait_limit(0, None) == rq.RESPIN_ERR_INVALID_ARG
+    assert rq.lib.respin_selftest_wait_limit(2000001, None) == rq.RESPIN_ERR_INVALID_ARG
+    assert "limit_us" in rq.last_error()

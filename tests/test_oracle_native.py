@@ -109,3 +109,40 @@ def test_gemm_equals_numpy_oracle_workload_rows():
     ref = O.w4a4_acc(qa, qw)
     assert np.array_equal(acc, ref)
     assert np.array_equal(out, O.w4a4_epilogue_bits(ref, sa, sw))
+
+
+def test_subspace_boundary_brute_force_tiny():
+    """D = 16, r = 4, stored subspace form: the three steps of zh §2.2 written
+    out as Python loops over the plan's rounded values."""
+    rs = np.random.default_rng(17)
+    D, r, n = 16, 4, 3
+    x = bits_of(rs.standard_normal((n, D)))
+    res = bits_of(rs.standard_normal((n, D)))
+    Q = np.linalg.qr(rs.standard_normal((D, r)))[0].astype(np.float32)
+    R = (np.eye(r) + 0.2 * rs.standard_normal((r, r))).astype(np.float32)
+    h64, hb, codes, scale = N.boundary_reference_subspace(x, res, Q, R)
+    Qq = O.round_to_bf16(Q)
+    M = [[float(np.float32(float(R[i, j]) - (1.0 if i == j else 0.0))) for j in range(r)] for i in range(r)]
+    xf, rf = O.bf16_bits_to_f32(x), O.bf16_bits_to_f32(res)
+    for t in range(n):
+        y = [sum(float(rf[t, d]) * float(Qq[d, j]) for d in range(D)) for j in range(r)]
+        z = [sum(y[j] * M[i][j] for j in range(r)) for i in range(r)]
+        for d in range(D):
+            want = float(xf[t, d]) + float(rf[t, d]) + sum(z[i] * float(Qq[d, i]) for i in range(r))
+            assert abs(h64[t, d] - want) <= 1e-13 * max(1.0, abs(want))
+    assert np.array_equal(hb, O.bf16_bits(h64))
+
+
+@pytest.mark.parametrize("name", ["tiny", "llama2_7b"])
+def test_subspace_native_matches_numpy(name):
+    fx = W.workload_fixture(name, N=24)
+    Qr, R = W.subspace_factors(fx.Q, fx.theta, fx.r)
+    Q32, R32 = Qr.astype(np.float32), R.astype(np.float32)
+    xb = O.bf16_bits(fx.x.float().numpy())
+    rb = O.bf16_bits(fx.residual.float().numpy())
+    a = N.boundary_reference_subspace(xb, rb, Q32, R32)
+    b = O.boundary_reference_subspace(fx.x.float().numpy(), fx.residual.float().numpy(), Q32, R32)
+    assert np.max(np.abs(a[0] - b[0])) <= 1e-12 * np.max(np.abs(b[0]))
+    assert np.array_equal(a[1], b[1])
+    assert np.array_equal(a[2], b[2])
+    assert np.array_equal(a[3].view(np.uint32), b[3].view(np.uint32))

@@ -382,3 +382,61 @@ def test_page_counts():
     assert round(on / 1e6, 1) == g["online_params_M"]
     tr = O.training_rotation_params(g["layers"], g["D"]) / 1e6
     assert round(tr + g["spinquant_training_params_M"], 1) == g["training_params_M"]
+
+
+# ---------------------------------------------------------------- subspace form (device Q-form plans)
+
+def test_subspace_row_form_equals_column_form():
+    # zh §2.2 steps 1-3 in the row form (y = res Q, z = y M^T, res + z Q^T)
+    # against the column-form function on the same vectors; the transposed
+    # transform and a dropped step fail.
+    D, r = 96, 12
+    rs = np.random.default_rng(21)
+    Q, _ = np.linalg.qr(rs.standard_normal((D, r)))
+    M = 0.1 * rs.standard_normal((r, r))
+    res, x = rs.standard_normal((5, D)), rs.standard_normal((5, D))
+    col = O.subspace_residual_rotation(res.T, Q, np.eye(r) + M).T + x
+    np.testing.assert_allclose(O.boundary_subspace_fp64(x, res, Q, M), col, atol=1e-13)
+    assert not np.allclose(O.boundary_subspace_fp64(x, res, Q, M.T), col, atol=1e-6)
+    assert not np.allclose(O.boundary_subspace_fp64(x, res, Q, np.zeros((r, r))), col, atol=1e-6)
+
+
+@pytest.mark.parametrize("D,k,nu", [(256, 8, 0.05), (512, 32, 1.0)])
+def test_subspace_fixture_exact_rank_equals_dense_T(D, k, nu):
+    # Exact rank (r = k): the fixture's stored form (Q_r, R_sub) reproduces the
+    # dense T = R_out^T R_in built independently through scipy's expm.
+    Q, th, T = _fixture(D, k, nu)
+    Qr, R = W.subspace_factors(Q, th, k)
+    rs = np.random.default_rng(22)
+    res, x = rs.standard_normal((6, D)), rs.standard_normal((6, D))
+    np.testing.assert_allclose(O.boundary_subspace_fp64(x, res, Qr, R - np.eye(k)),
+                               O.dense_boundary_fp64(x, res, T), atol=1e-12)
+    # and the rotation is orthogonal with det 1 (a product of plane rotations)
+    np.testing.assert_allclose(R.T @ R, np.eye(k), atol=1e-15)
+    assert abs(np.linalg.det(R) - 1.0) < 1e-12
+
+
+def test_subspace_plan_factors_round_once():
+    # M = R_sub - I is formed exactly and rounded once to binary32; Q is
+    # rounded to bfloat16. Hand-worked: 1 - 2^-24 (a float32) minus 1 is
+    # -2^-24, exact; -(1 - 2^-24) minus 1 = -(2 - 2^-24) rounds to -2 in
+    # binary32 (spacing 2^-22 below 2: 2^-24 away from -2, 3 2^-24 from the
+    # next value); 0.75 off the diagonal stays 0.75.
+    R = np.array([[1 - 2.0 ** -24, 0.75], [0.0, -(1 - 2.0 ** -24)]], np.float32)
+    Q = np.array([[1.0 + 2.0 ** -8, 0.3], [2.0 ** -20, -0.5]], np.float32)
+    Qq, M = O.subspace_plan_factors(Q, R)
+    assert M.tolist() == [[-2.0 ** -24, 0.75], [0.0, -2.0]]
+    assert Qq[0, 0] == 1.0          # 1 + 2^-8 is a bf16 tie: to even
+    assert Qq[1, 1] == -0.5
+    assert Qq[1, 0] == 2.0 ** -20
+
+
+def test_subspace_reference_matches_factor_form_on_fixture():
+    # With V = Qq M (no further rounding) the factor-form oracle gives the
+    # same h as the subspace-form oracle (different summation order only).
+    fx = W.workload_fixture("tiny")
+    Qr, R = W.subspace_factors(fx.Q, fx.theta, fx.r)
+    Qq, M = O.subspace_plan_factors(Qr.astype(np.float32), R.astype(np.float32))
+    x, res = fx.x.float().numpy(), fx.residual.float().numpy()
+    np.testing.assert_allclose(O.boundary_subspace_fp64(x, res, Qq, M),
+                               O.boundary_fp64(x, res, Qq, Qq @ M), rtol=0, atol=1e-12)

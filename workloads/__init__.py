@@ -201,6 +201,25 @@ def lowrank_factors(Q: np.ndarray, theta: np.ndarray, r: int):
     return U, V
 
 
+def subspace_factors(Q: np.ndarray, theta: np.ndarray, r: int):
+    """The stored subspace form (basis, rotation) of the same rank-r fix,
+    float64: ``Q_r`` = the first r columns of the plane basis and ``R_sub`` =
+    blockdiag of the 2x2 plane rotations [[cos t, -sin t], [sin t, cos t]],
+    so that ``R_sub - I`` = blockdiag(B_j)^T and ``Q_r (R_sub - I)`` equals
+    the ``V_r`` of :func:`lowrank_factors` (zh page §2.2 stores one D x r
+    basis and one r x r rotation per boundary)."""
+    if r % 2:
+        raise ValueError("r must be even so that no rotation plane is split")
+    m = r // 2
+    if m > len(theta):
+        raise ValueError("r larger than the rank of T - I")
+    R = np.eye(r)
+    for j in range(m):
+        c, s = math.cos(theta[j]), math.sin(theta[j])
+        R[2 * j:2 * j + 2, 2 * j:2 * j + 2] = [[c, -s], [s, c]]
+    return np.ascontiguousarray(Q[:, :r]), R
+
+
 @dataclass
 class BoundaryFixture:
     """Everything one boundary call needs, on the CPU."""
