@@ -90,6 +90,36 @@ respin_status_t respin_plan_create(respin_plan_t* out, int D, int r,
                                    const float* U_r, const float* V_r,
                                    unsigned flags);
 
+/*
+ * respin_plan_create_subspace -- prepare a boundary from the stored
+ * subspace form.
+ *
+ * Passage: zh §2.2 steps 1-3 keep, per boundary, one D x r basis Q and one
+ * r x r rotation R_sub and apply the fix as projection y = Q^T x, transform
+ * z = (R_sub - I) y inside the subspace, re-projection x + Q z; the online
+ * parameter count of zh §4 (64 D r) is this form. In the row convention of
+ * respin_boundary_forward the same fix is
+ *     y = residual Q,  z = y M^T,  h = residual + x + z Q^T,  M = R_sub - I,
+ * i.e. the factor form with U_r = Q and V_r = Q M, stored in half the bytes.
+ *
+ *   out    : receives the plan handle.
+ *   D      : hidden size; 2048 or 4096 (the two CTAs of a pair each hold
+ *            half of Q on chip).
+ *   r      : rank, 1 <= r <= 32.
+ *   Q      : HOST fp32 [D, r] row-major.
+ *   R_sub  : HOST fp32 [r, r] row-major.
+ *   flags  : 0, or RESPIN_H_FP32_DEBUG and/or RESPIN_ACT_INT3.
+ *
+ * The plan rounds Q to bfloat16 (round to nearest even) and forms
+ * M = R_sub - I exactly, rounded once to fp32; respin_boundary_forward then
+ * computes y and z in fp32 (z_i = sum_j y_j M_ij in j order) and h in fp32
+ * as for factor plans. Synchronous. Errors: INVALID_ARG, UNSUPPORTED, OOM,
+ * CUDA.
+ */
+respin_status_t respin_plan_create_subspace(respin_plan_t* out, int D, int r,
+                                            const float* Q, const float* R_sub,
+                                            unsigned flags);
+
 /* respin_plan_destroy -- free the plan's device factors. Waits for the device
  * to finish outstanding work first. Unknown or already destroyed handles give
  * INVALID_ARG. NULL is a no-op. */
@@ -112,7 +142,8 @@ respin_status_t respin_plan_destroy(respin_plan_t plan);
  * with B = 7 (INT4), or B = 3 for a plan made with RESPIN_ACT_INT3.
  * A token with amax < 2^-125 gets scale 0 and all-zero codes.
  *
- *   plan      : from respin_plan_create; its device must be current.
+ *   plan      : from respin_plan_create or respin_plan_create_subspace;
+ *               its device must be current.
  *   x         : bf16 [N, D] block output (device).
  *   residual  : bf16 [N, D] residual stream (device), or NULL for zero (then
  *               h' = x and the factors are not used).
@@ -203,6 +234,47 @@ respin_status_t respin_factors_from_subspace(int D, int r, const float* Q,
 respin_status_t respin_factors_from_transition(int D, int r, const float* T,
                                                double gap_tol, float* U_r,
                                                float* V_r, double* sigma);
+
+/*
+ * respin_fuse_weight -- fold the block rotations into a linear's weight.
+ *
+ * Passage: the rotations are merged into the weights offline so that the
+ * linears stay ordinary linears (zh §2.2, e.g. W~ = R^T W R; fr §2A,
+ * W~ = W R). For y = W x with the input arriving as x~ = R_in^T x and the
+ * output wanted as y~ = R_out^T y:
+ *     W_fused = R_out^T W R_in        (W_fused x~ = R_out^T W x),
+ * or W R_in when R_out is NULL.
+ *
+ *   O, K    : output and input size (O, K > 0).
+ *   W       : HOST fp32 [O, K] row-major (one row per output channel).
+ *   R_in    : HOST fp32 [K, K] row-major.
+ *   R_out   : HOST fp32 [O, O] row-major, or NULL.
+ *   W_fused : HOST fp32 [O, K] output (caller-owned).
+ * Host only: float64 products over the host's threads, each element one sum
+ * in a fixed order. Errors: INVALID_ARG, OOM.
+ */
+respin_status_t respin_fuse_weight(int O, int K, const float* W,
+                                   const float* R_in, const float* R_out,
+                                   float* W_fused);
+
+/*
+ * respin_quantize_weight -- per-output-channel symmetric INT4 (or INT3)
+ * weight codes for w4a4_gemm (the explainers evaluate W4A4 and W3A3, zh
+ * §3-§4; they give no weight quantizer). Per row o, in binary32 as for the
+ * activations: amax = max_k |W[o,k]|, inv = qmax / amax,
+ * q = clamp(rint(W[o,k] inv), -qmax-1, qmax) (ties to even),
+ * scale_w[o] = amax / qmax; a row with amax < 2^-125 gets scale 0 and zero
+ * codes.
+ *
+ *   O, K    : rows and columns (K even).
+ *   W       : HOST fp32 [O, K] row-major.
+ *   qmax    : 7 (INT4) or 3 (INT3).
+ *   q_w     : HOST uint8 [O, K/2] packed codes (element 2j in the low nibble).
+ *   scale_w : HOST fp32 [O].
+ * Host only. Errors: INVALID_ARG.
+ */
+respin_status_t respin_quantize_weight(int O, int K, const float* W, int qmax,
+                                       uint8_t* q_w, float* scale_w);
 
 /* respin_device_status -- synchronizes the current device, then returns and
  * clears the device status word through *code (0 = no kernel gave up; else

@@ -364,6 +364,26 @@ def boundary_reference_subspace(x, residual, Q32, R32, qmax: int = 7):
 
 
 # --------------------------------------------------------------------------
+# Offline weight preparation (zh §2.2 offline weight merging; fr §2A)
+# --------------------------------------------------------------------------
+
+def fuse_weight_fp64(W, R_in, R_out=None) -> np.ndarray:
+    """W~ = R_out^T W R_in (or W R_in), float64: for y = W x with x~ = R_in^T x,
+    W~ x~ = R_out^T y."""
+    Wf = np.asarray(W, np.float64) @ np.asarray(R_in, np.float64)
+    if R_out is not None:
+        Wf = np.asarray(R_out, np.float64).T @ Wf
+    return Wf
+
+
+def quantize_weight_rows(W32, qmax: int = 7):
+    """Per-output-channel symmetric codes of float32 W [O, K]: the activation
+    quantizer applied to each row (binary32), packed two per byte."""
+    codes, scale = quantize_per_token(np.asarray(W32, np.float32), qmax)
+    return pack_int4(codes), scale
+
+
+# --------------------------------------------------------------------------
 # Counts the pages print (zh §4; nl §4; es §4; fr §4)
 # --------------------------------------------------------------------------
 

@@ -26,9 +26,10 @@ RESPIN_H_FP32_DEBUG = 1
 RESPIN_ACT_INT3 = 2
 
 # Every entry point include/respin.h declares (checked by the tests).
-EXPORTED = ("respin_plan_create", "respin_plan_destroy",
+EXPORTED = ("respin_plan_create", "respin_plan_create_subspace", "respin_plan_destroy",
             "respin_boundary_forward", "w4a4_gemm", "w4a4_gemm_i32",
             "respin_factors_from_subspace", "respin_factors_from_transition",
+            "respin_fuse_weight", "respin_quantize_weight",
             "respin_device_status", "respin_selftest_wait_limit",
             "respin_last_error", "respin_version")
 
@@ -51,6 +52,7 @@ def _load() -> ctypes.CDLL:
     vp, i32, u32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_uint
     fp = ctypes.POINTER(ctypes.c_float)
     lib.respin_plan_create.argtypes = [ctypes.POINTER(vp), i32, i32, fp, fp, u32]
+    lib.respin_plan_create_subspace.argtypes = [ctypes.POINTER(vp), i32, i32, fp, fp, u32]
     lib.respin_plan_destroy.argtypes = [vp]
     lib.respin_boundary_forward.argtypes = [vp, vp, vp, i32, vp, vp, vp, vp]
     lib.w4a4_gemm.argtypes = [vp, vp, vp, vp, i32, i32, i32, vp, vp]
@@ -58,6 +60,8 @@ def _load() -> ctypes.CDLL:
     dp = ctypes.POINTER(ctypes.c_double)
     lib.respin_factors_from_subspace.argtypes = [i32, i32, fp, fp, fp, fp]
     lib.respin_factors_from_transition.argtypes = [i32, i32, fp, ctypes.c_double, fp, fp, dp]
+    lib.respin_fuse_weight.argtypes = [i32, i32, fp, fp, fp, fp]
+    lib.respin_quantize_weight.argtypes = [i32, i32, fp, i32, vp, fp]
     lib.respin_device_status.argtypes = [ctypes.POINTER(ctypes.c_int)]
     lib.respin_selftest_wait_limit.argtypes = [u32, vp]
     for name in EXPORTED[:-2]:
@@ -127,8 +131,29 @@ class Plan:
             pass
 
 
+class SubspacePlan(Plan):
+    """respin_plan_create_subspace: a boundary from its stored subspace form
+    (host fp32 basis Q [D, r] and rotation R_sub [r, r])."""
+
+    def __init__(self, D: int, r: int, Q, R_sub, flags: int = 0):
+        self.D, self.r, self.flags = int(D), int(r), int(flags)
+        self.handle = ctypes.c_void_p()
+        fp = ctypes.POINTER(ctypes.c_float)
+        Qa = np.ascontiguousarray(Q, dtype=np.float32)
+        Ra = np.ascontiguousarray(R_sub, dtype=np.float32)
+        if Qa.shape != (self.D, self.r) or Ra.shape != (self.r, self.r):
+            raise ValueError("Q must be [D, r] and R_sub [r, r]")
+        _check(lib.respin_plan_create_subspace(ctypes.byref(self.handle), self.D, self.r,
+                                               Qa.ctypes.data_as(fp), Ra.ctypes.data_as(fp),
+                                               self.flags))
+
+
 def respin_plan_create(D, r, U_r=None, V_r=None, flags=0) -> Plan:
     return Plan(D, r, U_r, V_r, flags)
+
+
+def respin_plan_create_subspace(D, r, Q, R_sub, flags=0) -> SubspacePlan:
+    return SubspacePlan(D, r, Q, R_sub, flags)
 
 
 def respin_plan_destroy(plan: Plan) -> None:
@@ -204,6 +229,33 @@ def respin_factors_from_transition(T, r: int, gap_tol: float = 1e-6):
                                               U.ctypes.data_as(fp), V.ctypes.data_as(fp),
                                               sig.ctypes.data_as(ctypes.POINTER(ctypes.c_double))))
     return U, V, sig
+
+
+def respin_fuse_weight(W, R_in, R_out=None):
+    """W_fused = R_out^T W R_in (or W R_in) for host fp32 arrays W [O, K],
+    R_in [K, K], R_out [O, O]; float64 products on the host."""
+    W = np.ascontiguousarray(W, dtype=np.float32)
+    O, K = W.shape
+    Ri = _host_f32(R_in, (K, K), "R_in")
+    Ro = None if R_out is None else _host_f32(R_out, (O, O), "R_out")
+    fp = ctypes.POINTER(ctypes.c_float)
+    out = np.empty((O, K), np.float32)
+    _check(lib.respin_fuse_weight(O, K, W.ctypes.data_as(fp), Ri.ctypes.data_as(fp),
+                                  None if Ro is None else Ro.ctypes.data_as(fp), out.ctypes.data_as(fp)))
+    return out
+
+
+def respin_quantize_weight(W, qmax: int = 7):
+    """(packed codes uint8 [O, K/2], scales fp32 [O]) of host fp32 W [O, K],
+    symmetric per output channel (qmax 7: INT4, 3: INT3)."""
+    W = np.ascontiguousarray(W, dtype=np.float32)
+    O, K = W.shape
+    q = np.empty((O, K // 2), np.uint8)
+    sc = np.empty(O, np.float32)
+    fp = ctypes.POINTER(ctypes.c_float)
+    _check(lib.respin_quantize_weight(O, K, W.ctypes.data_as(fp), int(qmax), q.ctypes.data,
+                                      sc.ctypes.data_as(fp)))
+    return q, sc
 
 
 def respin_selftest_wait_limit(limit_us: int, stream=None) -> None:

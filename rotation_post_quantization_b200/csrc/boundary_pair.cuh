@@ -1,0 +1,439 @@
+// Pair boundary kernel: the stored subspace form of the basis fix (one D x r
+// basis Q and one r x r transform M = R_sub - I per boundary, the ReSpinQuant
+// explainers' zh page §2.2 steps 1-3, row convention) fused with per-token
+// INT4 / INT3 quantization (zh §3-§4):
+//   y = residual Q ; z = y M^T ; h = (residual + x) + z Q^T   (fp32)
+//   h' = bf16(h) ; amax = max|h'| ; inv = qmax/amax ; q = rint(h' inv)
+//
+// Design (B200, one CTA per SM, CTA pairs = clusters of 2, 8 warps):
+//  * The two CTAs of a pair split the D columns: CTA c owns the DC = D/2
+//    columns [c DC, (c+1) DC) of every token; warp w owns DC/8 of them
+//    (NB blocks of 64) in every phase, so each shared-memory buffer block is
+//    private to one warp, which refills it as soon as it is done with it.
+//  * A round is one tile of T <= 16 tokens (one m16 tile; the host picks T so
+//    that every pair gets the same number of rounds). Residual tiles arrive
+//    by 2-D tensor copies (box 64 columns x 16 rows, 128-byte swizzle) into
+//    two buffers and x tiles into a third; the first two residual tiles and
+//    the first x tile are requested at launch, x of round r+1 when a warp's
+//    re-projection of round r is done, the residual of round r+2 when its
+//    codes are written. h' is written back over the residual.
+//  * Both products run on mma.sync m16n8k16 (bf16, fp32 accumulate), tokens
+//    on the M side. Q is read from global memory (L2-resident, shared by all
+//    CTAs) as pre-arranged fragments, one 16-byte load per lane per fragment
+//    group, one 64-column block ahead in registers: the projection's B
+//    fragments (pairs along the column) and the re-projection's (pairs along
+//    r, columns permuted so that each lane's outputs are two 16-byte chunks
+//    of a row). z is split into bf16 hi + lo parts.
+//  * The two whole-row dependencies (y needs every column, amax needs every
+//    column) are exchanged by pushing this CTA's partials into the peer's
+//    shared memory with st.async (completion counted on the peer's mbarrier,
+//    polled with a non-blocking test). Partial sums are combined in rank
+//    order, so both CTAs use the identical y and z.
+//  * Every wait is bounded; after a wait gave up the CTA stores nothing more
+//    and requests no further tensor copies (those in flight are waited for).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "boundary_kernels.cuh"
+#include "boundary_rowtile.cuh"
+#include "ptx.cuh"
+
+namespace respin {
+
+constexpr int kPrR = 32;          // padded rank of the pair kernel
+constexpr int kPrT = 16;          // token slots per round (one m16 tile)
+constexpr int kPrThreads = 256;   // 8 warps
+constexpr int kPrBlockBytes = kPrT * 128;   // one 64-column block of a 16-row tile
+
+// Column (within a 64-column block) of output column n of re-projection n8
+// tile t: lane (g, q) then owns columns 8q..8q+7 (tiles 0-3) and
+// 32+8q..32+8q+7 (tiles 4-7), two 16-byte chunks of every token row.
+__host__ __device__ constexpr int pr_channel(int t, int n) {
+  return 32 * (t >> 2) + 8 * (n >> 1) + 2 * (t & 3) + (n & 1);
+}
+
+template <int DC>
+struct PrCfg {
+  static_assert(DC == 1024 || DC == 2048, "columns per CTA");
+  static constexpr int NB = DC / 512;                          // 64-column blocks per warp
+  static constexpr uint32_t kTileBytes = kPrT * DC * 2;        // one 16-row tile
+  static constexpr int YP = 40;                                // z row pitch (floats)
+  static constexpr int BP = 33;                                // y / M row pitch (floats)
+  static constexpr uint32_t oRes = 0;                          // 2 residual tiles (h' in place)
+  static constexpr uint32_t oX = 2 * kTileBytes;               // x tile
+  static constexpr uint32_t oYpart = 3 * kTileBytes;           // [8][16][32] partial y, swizzled
+  static constexpr uint32_t oYpeer = oYpart + 8 * kPrT * kPrR * 4;   // [2][16][32] peer's partial y
+  static constexpr uint32_t oY = oYpeer + 2 * kPrT * kPrR * 4;       // [16][BP] full y
+  static constexpr uint32_t oZ = oY + kPrT * BP * 4;                 // [16][YP] z
+  static constexpr uint32_t oM = oZ + kPrT * YP * 4;                 // [32][BP] M
+  static constexpr uint32_t oWamax = oM + kPrR * BP * 4;             // [8][16]
+  static constexpr uint32_t oApeer = oWamax + 8 * kPrT * 4;          // [2][16] peer's row maxima
+  static constexpr uint32_t oRinv = oApeer + 2 * kPrT * 4;           // [16]
+  static constexpr uint32_t oBars = oRinv + kPrT * 4;  // rbar[8][2], xbar[8], ybar[2], abar[2]
+  static constexpr uint32_t kSmem = oBars + 28 * 8 + 1024;           // + alignment slack
+  static_assert(oBars % 8 == 0 && oX % 1024 == 0 && kTileBytes % 1024 == 0, "alignment");
+};
+
+// Asynchronous 8- / 4-byte stores into a peer CTA's shared memory; their bytes
+// complete a transaction count on the peer's mbarrier (both addresses are
+// shared::cluster addresses).
+__device__ __forceinline__ void st_async_f32x2(uint32_t raddr, float a, float b, uint32_t rbar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [%0], {%1, %2}, [%3];" ::"r"(raddr),
+               "f"(a), "f"(b), "r"(rbar)
+               : "memory");
+}
+__device__ __forceinline__ void st_async_f32(uint32_t raddr, float a, uint32_t rbar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(raddr),
+               "r"(__float_as_uint(a)), "r"(rbar)
+               : "memory");
+}
+
+// tmR / tmX: bf16 [N, D] residual / x, box {64 columns, 16 rows}, 128-byte
+// swizzle. Pf / Rf: the plan's projection / re-projection fragments of both
+// column halves (pr_pack_frags), 8 uint4 per lane per 64-column block.
+// Mg: M = R_sub - I, fp32 [32][32] row-major (zero padded).
+template <int DC, bool F32OUT>
+__global__ void __launch_bounds__(kPrThreads, 1)
+boundary_pair_kernel(const __grid_constant__ CUtensorMap tmR, const __grid_constant__ CUtensorMap tmX,
+                     const uint4* __restrict__ Pf, const uint4* __restrict__ Rf, const float* __restrict__ Mg,
+                     int N, int D, int T, void* __restrict__ h_out, uint8_t* __restrict__ q_out,
+                     float* __restrict__ scale_out, float qmax) {
+  using C = PrCfg<DC>;
+  constexpr int NB = C::NB, YP = C::YP, BP = C::BP;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (base - raw);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, q4 = lane & 3;
+  const uint32_t rank = cluster_ctarank(), peer = rank ^ 1u;
+  const int cid = static_cast<int>(cluster_id_x()), ncl = static_cast<int>(ncluster_x());
+  const int ntiles = (N + T - 1) / T;
+  const int rounds = cid < ntiles ? (ntiles - cid + ncl - 1) / ncl : 0;
+  const int col0 = static_cast<int>(rank) * DC;
+  const int b0 = warp * NB;                         // this warp's first block
+
+  float* ypart = reinterpret_cast<float*>(smem + C::oYpart);
+  const float* ypeer = reinterpret_cast<const float*>(smem + C::oYpeer);
+  float* ybuf = reinterpret_cast<float*>(smem + C::oY);
+  float* zbuf = reinterpret_cast<float*>(smem + C::oZ);
+  float* msm = reinterpret_cast<float*>(smem + C::oM);
+  float* wamax = reinterpret_cast<float*>(smem + C::oWamax);
+  const float* apeer = reinterpret_cast<const float*>(smem + C::oApeer);
+  float* rowinv = reinterpret_cast<float*>(smem + C::oRinv);
+  const uint32_t bars = base + C::oBars;
+  auto rbar = [&](int b) { return bars + 16 * warp + 8 * b; };
+  const uint32_t xbar = bars + 128 + 8 * warp;
+  auto ybar = [&](int p) { return bars + 192 + 8 * p; };
+  auto abar = [&](int p) { return bars + 208 + 8 * p; };
+  const uint4* pf = Pf + static_cast<size_t>(rank) * (DC / 64) * 8 * 32 + lane;   // this half's fragments
+  const uint4* rf = Rf + static_cast<size_t>(rank) * (DC / 64) * 8 * 32 + lane;
+
+  if (lane == 0) {
+    mbar_init(rbar(0), 1);
+    mbar_init(rbar(1), 1);
+    mbar_init(xbar, 1);
+    if (warp == 0)
+      for (int p = 0; p < 2; ++p) { mbar_init(ybar(p), 1); mbar_init(abar(p), 1); }
+    fence_mbarrier_init();
+    if (warp == 0) {
+      asm volatile("prefetch.tensormap [%0];" ::"l"(&tmR) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"(&tmX) : "memory");
+    }
+  }
+  __syncthreads();
+  // the peer may push into this CTA only after its barriers exist; the
+  // matching wait precedes this CTA's first push
+  cluster_arrive();
+
+  // Tensor copies of this warp's blocks (one lane per block). All buffers are
+  // private to the warp: warp w alone reads and writes the columns of its
+  // blocks, so it refills them as soon as it is done with them.
+  bool res_pend0 = false, res_pend1 = false, x_pend = false;
+  auto issue_res = [&](int r) {   // round r's residual into buffer r & 1
+    const int rb = r & 1;
+    if (lane == 0) mbar_arrive_expect_tx(rbar(rb), NB * kPrBlockBytes);
+    __syncwarp();
+    if (lane < NB)
+      tma_load_2d(base + C::oRes + rb * C::kTileBytes + (b0 + lane) * kPrBlockBytes, &tmR, col0 + (b0 + lane) * 64,
+                  (cid + r * ncl) * T, rbar(rb));
+    if (rb) res_pend1 = true; else res_pend0 = true;
+  };
+  auto issue_x = [&](int r) {
+    if (lane == 0) mbar_arrive_expect_tx(xbar, NB * kPrBlockBytes);
+    __syncwarp();
+    if (lane < NB)
+      tma_load_2d(base + C::oX + (b0 + lane) * kPrBlockBytes, &tmX, col0 + (b0 + lane) * 64, (cid + r * ncl) * T,
+                  xbar);
+    x_pend = true;
+  };
+  if (rounds > 0) { issue_res(0); issue_x(0); }
+  if (rounds > 1) issue_res(1);
+  for (int i = tid; i < kPrR * kPrR; i += kPrThreads) msm[(i >> 5) * BP + (i & 31)] = __ldg(Mg + i);
+
+  const int arow = (lane & 7) + 8 * ((lane >> 3) & 1);   // ldmatrix A row
+  bool ok = true;
+  bool cluster_waited = false;
+  for (int r = 0; r < rounds; ++r) {
+    const int tile = cid + r * ncl, row0 = tile * T;
+    const int rb = r & 1, par = r & 1;
+    const uint32_t upar = static_cast<uint32_t>(r >> 1) & 1u;
+    const uint32_t sRes = base + C::oRes + rb * C::kTileBytes;
+    uint8_t* resp = smem + C::oRes + rb * C::kTileBytes;
+    if (tid == 0) {
+      mbar_arrive_expect_tx(ybar(par), kPrT * kPrR * 4);
+      mbar_arrive_expect_tx(abar(par), kPrT * 4);
+    }
+
+    // ---- projection: this warp's partial y over its NB blocks
+    uint4 fr[2][8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) fr[0][i] = __ldg(pf + (b0 * 8 + i) * 32);
+    if (rb ? res_pend1 : res_pend0) {
+      ok = mbar_wait(rbar(rb), static_cast<uint32_t>(r >> 1) & 1u, kSitePairLoad) && ok;
+      if (rb) res_pend1 = false; else res_pend0 = false;
+    }
+    ok = __all_sync(0xffffffffu, ok);
+    float acc1[4][4];
+#pragma unroll
+    for (int p = 0; p < 4; ++p) acc1[p][0] = acc1[p][1] = acc1[p][2] = acc1[p][3] = 0.f;
+#pragma unroll
+    for (int j = 0; j < NB; ++j) {
+      if (j + 1 < NB) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) fr[(j + 1) & 1][i] = __ldg(pf + ((b0 + j + 1) * 8 + i) * 32);
+      }
+      const uint32_t blk = sRes + (b0 + j) * kPrBlockBytes;
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        uint32_t a[4];
+        ldmatrix_x4(blk + sw128(arow, 2 * kk + (lane >> 4)), a[0], a[1], a[2], a[3]);
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+          const uint4& v = fr[j & 1][kk * 2 + (p >> 1)];
+          mma_bf16_16816(acc1[p], a, u4c(v, 2 * (p & 1)), u4c(v, 2 * (p & 1) + 1));
+        }
+      }
+    }
+    // first re-projection fragments load while y is exchanged
+#pragma unroll
+    for (int i = 0; i < 8; ++i) fr[0][i] = __ldg(rf + (b0 * 8 + i) * 32);
+    {
+      // partial y of this warp: element (tok, r) at tok * 32 + (r ^ 8 (tok & 3))
+      float* yp = ypart + warp * kPrT * kPrR;
+#pragma unroll
+      for (int p = 0; p < 4; ++p) {
+        const int c = 8 * (p ^ (g & 3)) + 2 * q4;
+        *reinterpret_cast<float2*>(yp + g * kPrR + c) = make_float2(acc1[p][0], acc1[p][1]);
+        *reinterpret_cast<float2*>(yp + (g + 8) * kPrR + c) = make_float2(acc1[p][2], acc1[p][3]);
+      }
+    }
+    ok = __syncthreads_and(ok) != 0;
+
+    // ---- y over the pair: thread t owns token t/16, r = 2 (t%16), +1; its
+    // partial (warps summed in order) goes to the peer
+    const int yt = tid >> 4, yc = 2 * (tid & 15);
+    float2 ys = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+      const float2 v =
+          *reinterpret_cast<const float2*>(ypart + (w * kPrT + yt) * kPrR + (yc ^ (8 * (yt & 3))));
+      ys.x += v.x;
+      ys.y += v.y;
+    }
+    if (!cluster_waited) { cluster_wait(); cluster_waited = true; }
+    st_async_f32x2(map_to_rank(base + C::oYpeer + ((par * kPrT + yt) * kPrR + yc) * 4, peer), ys.x, ys.y,
+                   map_to_rank(ybar(par), peer));
+    ok = mbar_spin_cluster(ybar(par), upar, kSitePairPeer) && ok;
+    {
+      const float2 v = *reinterpret_cast<const float2*>(ypeer + (par * kPrT + yt) * kPrR + yc);
+      const float2 y = rank == 0 ? make_float2(ys.x + v.x, ys.y + v.y) : make_float2(v.x + ys.x, v.y + ys.y);
+      ybuf[yt * BP + yc] = y.x;
+      ybuf[yt * BP + yc + 1] = y.y;
+    }
+    __syncwarp();   // the 16 threads of a token share a warp
+    {
+      // z[t][i] = sum_j y[t][j] M[i][j] (j in order), i = yc, yc + 1
+      float z0 = 0.f, z1 = 0.f;
+      const float* yrow = ybuf + yt * BP;
+#pragma unroll
+      for (int jj = 0; jj < kPrR; ++jj) {
+        const float yv = yrow[jj];
+        z0 = __fmaf_rn(yv, msm[yc * BP + jj], z0);
+        z1 = __fmaf_rn(yv, msm[(yc + 1) * BP + jj], z1);
+      }
+      *reinterpret_cast<float2*>(zbuf + yt * YP + yc) = make_float2(z0, z1);
+    }
+    ok = __syncthreads_and(ok) != 0;
+
+    // ---- re-projection: h = (residual + x) + z Q^T over this warp's blocks
+    uint32_t ahi[2][4], alo[2][4];
+#pragma unroll
+    for (int kk = 0; kk < 2; ++kk) {
+      const float* z0 = zbuf + g * YP + 16 * kk + 2 * q4;
+      split_bf16x2(*reinterpret_cast<const float2*>(z0), ahi[kk][0], alo[kk][0]);
+      split_bf16x2(*reinterpret_cast<const float2*>(z0 + 8 * YP), ahi[kk][1], alo[kk][1]);
+      split_bf16x2(*reinterpret_cast<const float2*>(z0 + 8), ahi[kk][2], alo[kk][2]);
+      split_bf16x2(*reinterpret_cast<const float2*>(z0 + 8 * YP + 8), ahi[kk][3], alo[kk][3]);
+    }
+    if (x_pend) {
+      ok = mbar_wait(xbar, static_cast<uint32_t>(r) & 1u, kSitePairLoad) && ok;
+      x_pend = false;
+    }
+    ok = __all_sync(0xffffffffu, ok);
+    uint32_t amax2[2] = {0u, 0u};   // running max |h'| (bf16x2) of rows g and g + 8
+#pragma unroll
+    for (int j = 0; j < NB; ++j) {
+      if (j + 1 < NB) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) fr[(j + 1) & 1][i] = __ldg(rf + ((b0 + j + 1) * 8 + i) * 32);
+      }
+      const int b = b0 + j;
+      float acc[8][4];
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk) {
+          const uint4& v = fr[j & 1][t];
+          const uint32_t bb0 = u4c(v, 2 * kk), bb1 = u4c(v, 2 * kk + 1);
+          mma_bf16_16816(acc[t], ahi[kk], bb0, bb1);
+          mma_bf16_16816(acc[t], alo[kk], bb0, bb1);
+        }
+      }
+      const uint8_t* rblk = resp + b * kPrBlockBytes;
+      const uint8_t* xblk = smem + C::oX + b * kPrBlockBytes;
+      // epilogue: row g + 8 hh, chunk c = columns 32 c + 8 q .. + 7 (tiles
+      // 4 c .. 4 c + 3, word i = tile 4 c + i); odd g loads chunk 1 first
+      // (conflict-free 16-byte shared loads)
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int row = g + 8 * hh;
+        const bool store = ok && row < T && row0 + row < N;
+        const size_t grow = static_cast<size_t>(store ? row0 + row : 0);
+        const uint32_t oa = sw128(row, 4 * (g & 1) + q4), ob = sw128(row, 4 * (1 - (g & 1)) + q4);
+        const uint4 ra = *reinterpret_cast<const uint4*>(rblk + oa);
+        const uint4 rb_ = *reinterpret_cast<const uint4*>(rblk + ob);
+        const uint4 xa = *reinterpret_cast<const uint4*>(xblk + oa);
+        const uint4 xb = *reinterpret_cast<const uint4*>(xblk + ob);
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const bool first = c == (g & 1);
+          const uint4 rv = first ? ra : rb_, xv = first ? xa : xb;
+          const uint32_t so = first ? oa : ob;
+          const uint32_t rw[4] = {rv.x, rv.y, rv.z, rv.w}, xw[4] = {xv.x, xv.y, xv.z, xv.w};
+          uint32_t hw[4];
+          float2 hf[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int t = 4 * c + i;
+            const float2 sum = add_f32x2(bf16x2_to_f32x2(rw[i]), bf16x2_to_f32x2(xw[i]));
+            hf[i] = add_f32x2(sum, make_float2(acc[t][2 * hh], acc[t][2 * hh + 1]));
+            hw[i] = pack_bf16x2(hf[i].x, hf[i].y);
+            amax2[hh] = absmax_bf16x2(amax2[hh], hw[i]);
+          }
+          const uint4 hv = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+          *reinterpret_cast<uint4*>(resp + b * kPrBlockBytes + so) = hv;
+          const int gcol = col0 + b * 64 + 32 * c + 8 * q4;
+          if (store && h_out != nullptr) {
+            if constexpr (F32OUT) {
+              float4* hp = reinterpret_cast<float4*>(static_cast<float*>(h_out) + grow * D + gcol);
+              hp[0] = make_float4(hf[0].x, hf[0].y, hf[1].x, hf[1].y);
+              hp[1] = make_float4(hf[2].x, hf[2].y, hf[3].x, hf[3].y);
+            } else {
+              *reinterpret_cast<uint4*>(static_cast<bf16*>(h_out) + grow * D + gcol) = hv;
+            }
+          }
+        }
+      }
+    }
+    // this warp's x blocks are read: the next round's x
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (ok && r + 1 < rounds) issue_x(r + 1);
+
+    // ---- row amax over the warps, then over the pair
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      float m = fmaxf(bf16_lo_f32(amax2[hh]), bf16_hi_f32(amax2[hh]));
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+      if (q4 == 0) wamax[warp * kPrT + g + 8 * hh] = m;
+    }
+    ok = __syncthreads_and(ok) != 0;
+    if (tid < kPrT) {
+      float m = 0.f;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) m = fmaxf(m, wamax[w * kPrT + tid]);
+      st_async_f32(map_to_rank(base + C::oApeer + (par * kPrT + tid) * 4, peer), m, map_to_rank(abar(par), peer));
+      ok = mbar_spin_cluster(abar(par), upar, kSitePairPeer) && ok;
+      m = fmaxf(m, apeer[par * kPrT + tid]);
+      float inv, sc;
+      inv_and_scale(m, qmax, inv, sc);
+      rowinv[tid] = inv;
+      if (ok && rank == 0 && tid < T && row0 + tid < N) scale_out[row0 + tid] = sc;
+    }
+    ok = __syncthreads_and(ok) != 0;
+
+    // ---- codes of this warp's columns from h' in shared memory: lane l of
+    // step s takes chunk (32 s + l) of the warp's 16 rows x 8 NB chunks
+    constexpr int kRowChunks = 8 * NB;
+#pragma unroll 4
+    for (int s = 0; s < kPrT * kRowChunks / 32; ++s) {
+      const int k = 32 * s + lane;
+      const int tok = k / kRowChunks, cc = k % kRowChunks;
+      const int b = b0 + (cc >> 3);
+      const uint4 hv = *reinterpret_cast<const uint4*>(resp + b * kPrBlockBytes + sw128(tok, cc & 7));
+      const uint32_t code = quantize8_x2(hv, rowinv[tok]);
+      if (ok && tok < T && row0 + tok < N)
+        reinterpret_cast<uint32_t*>(q_out)[(static_cast<size_t>(row0 + tok) * D + col0 + 64 * b + 8 * (cc & 7)) / 8] =
+            code;
+    }
+    // this warp's residual blocks are read: round r + 2's residual
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (ok && r + 2 < rounds) issue_res(r + 2);
+  }
+  if (!cluster_waited) cluster_wait();   // no round: close the set-up barrier phase
+  // neither CTA may leave while the peer can still push into it
+  cluster_sync();
+}
+
+// Host side: the plan's Q fragments for boundary_pair_kernel<D/2>. Qb: bf16
+// bits of Q, [D][rr] row-major (rr <= 32, zero padded to 32 here). For column
+// half c and its 64-column block b (columns d0 = c D/2 + 64 b ..), lane
+// (g, q) gets 8 uint4 per block:
+//   projection (Pf): register i = 2 (4 kk + p) + e holds (Q[d][n], Q[d+1][n])
+//     with d = d0 + 16 kk + 2q + 8e, n = 8p + g;
+//   re-projection (Rf): register i = 2 (2 t + kk) + e holds (Q[d][m], Q[d][m+1])
+//     with d = d0 + pr_channel(t, g), m = 16 kk + 2q + 8e;
+// stored at uint4 ((c D/128 + b) 8 + i/4) 32 + lane, component i % 4.
+inline void pr_pack_frags(const uint16_t* Qb, int D, int rr, uint32_t* Pf, uint32_t* Rf) {
+  auto q = [&](int d, int r) -> uint32_t {
+    return r < rr ? Qb[static_cast<size_t>(d) * rr + r] : 0u;
+  };
+  const int nblk = D / 64;   // blocks of both halves, in order
+  for (int bb = 0; bb < nblk; ++bb)
+    for (int lane = 0; lane < 32; ++lane) {
+      const int g = lane >> 2, qq = lane & 3;
+      const int d0 = 64 * bb;
+      for (int i = 0; i < 32; ++i) {
+        const size_t idx = ((static_cast<size_t>(bb) * 8 + i / 4) * 32 + lane) * 4 + i % 4;
+        {
+          const int e = i & 1, p = (i >> 1) & 3, kk = i >> 3;
+          const int d = d0 + 16 * kk + 2 * qq + 8 * e, n = 8 * p + g;
+          Pf[idx] = q(d, n) | (q(d + 1, n) << 16);
+        }
+        {
+          const int e = i & 1, kk = (i >> 1) & 1, t = i >> 2;
+          const int d = d0 + pr_channel(t, g), m = 16 * kk + 2 * qq + 8 * e;
+          Rf[idx] = q(d, m) | (q(d, m + 1) << 16);
+        }
+      }
+    }
+}
+
+}  // namespace respin

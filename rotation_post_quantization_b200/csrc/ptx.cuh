@@ -114,6 +114,36 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t par
   return ok != 0;
 }
 
+// Non-blocking test with acquire semantics at cluster scope.
+__device__ __forceinline__ bool mbar_test_wait_cluster(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Wait for a phase that a PEER CTA completes (st.async transaction bytes),
+// by polling with the non-blocking test: a thread suspended in try_wait was
+// measured on B200 to sleep for microseconds past a completion signalled
+// from another SM. Bounded like mbar_wait.
+__device__ __forceinline__ bool mbar_spin_cluster(uint32_t bar, uint32_t parity, int site,
+                                                  uint64_t limit_ns = kWaitLimitNs) {
+  if (mbar_test_wait_cluster(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  while (true) {
+    if (mbar_test_wait_cluster(bar, parity)) return true;
+    if (globaltimer() - t0 > limit_ns) {
+      record_status(site);
+      return false;
+    }
+  }
+}
+
 __device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity, int site,
                                                   uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait_cluster(bar, parity)) return true;

@@ -20,8 +20,10 @@
 #include "respin.h"
 #include "ptx.cuh"
 #include "boundary_kernels.cuh"
+#include "boundary_pair.cuh"
 #include "boundary_rowtile.cuh"
 #include "factor_builder.h"
+#include "weight_tool.h"
 #include "w4a4_gemm_kernels.cuh"
 #include "w4a4_gemm_skinny.cuh"
 
@@ -94,6 +96,13 @@ struct respin_plan_s {
   bool has_tiny = false;
   __nv_bfloat16* factors_tiny = nullptr;
   BoundaryConfig cfg_tiny;
+  // Plans made from the stored subspace form (Q, R_sub): the pair kernel.
+  bool subspace = false;
+  uint32_t* q_pair = nullptr;    // projection then re-projection fragments of Q (pr_pack_frags)
+  float* m_pair = nullptr;       // M = R_sub - I, fp32 [32][32]
+  const void* pair_fn = nullptr;
+  size_t pair_smem = 0;
+  int pair_max = 0;              // co-resident CTA pairs
 };
 
 // Calls with at most this many tokens use cfg_small when the plan has one
@@ -139,14 +148,14 @@ static EncodeTiledFn encode_tiled() {
 }
 
 // 2-D bf16 tensor map over a row-major [rows, cols] matrix with a box of
-// 16 rows x 64 columns (128 bytes) in the 128-byte swizzle; rows past the end
-// read as zeros.
-bool make_tmap_bf16_tile(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols) {
+// box_rows rows x 64 columns (128 bytes) in the 128-byte swizzle; rows past
+// the end read as zeros.
+bool make_tmap_bf16_tile(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows = kRtT) {
   EncodeTiledFn fn = encode_tiled();
   if (!fn) return false;
   const cuuint64_t dims[2] = {cols, rows};
   const cuuint64_t strides[1] = {cols * 2};
-  const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(kRtT)};
+  const cuuint32_t box[2] = {64, box_rows};
   const cuuint32_t estr[2] = {1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
@@ -319,6 +328,28 @@ respin_status_t configure_boundary(int D, int R, bool f32, BoundaryConfig* out, 
               "no cluster configuration holds the factor slices for D=%d, padded r=%d", D, R);
 }
 
+template <int DC, bool F32>
+const void* pair_fn() {
+  return reinterpret_cast<const void*>(&boundary_pair_kernel<DC, F32>);
+}
+
+// The pair kernel for D columns (D / 2 per CTA) and its co-resident pairs.
+respin_status_t configure_pair(int D, bool f32, respin_plan_s* p) {
+  const int DC = D / 2;
+  const void* fn = nullptr;
+  size_t smem = 0;
+  if (DC == 1024) { fn = f32 ? pair_fn<1024, true>() : pair_fn<1024, false>(); smem = PrCfg<1024>::kSmem; }
+  if (DC == 2048) { fn = f32 ? pair_fn<2048, true>() : pair_fn<2048, false>(); smem = PrCfg<2048>::kSmem; }
+  if (fn == nullptr)
+    return fail(RESPIN_ERR_UNSUPPORTED, "subspace plans need D in {2048, 4096} (got D=%d)", D);
+  const int n = max_active_clusters(fn, 2, smem, kPrThreads);
+  if (n <= 0) return fail(RESPIN_ERR_UNSUPPORTED, "the pair kernel (%zu bytes of shared memory) cannot be launched", smem);
+  p->pair_fn = fn;
+  p->pair_smem = smem;
+  p->pair_max = n;
+  return ok();
+}
+
 respin_status_t check_device(int want) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
@@ -466,6 +497,62 @@ respin_status_t respin_plan_create(respin_plan_t* out, int D, int r, const float
   return ok();
 }
 
+respin_status_t respin_plan_create_subspace(respin_plan_t* out, int D, int r, const float* Q,
+                                            const float* R_sub, unsigned flags) {
+  t_last_error.clear();
+  if (out == nullptr) return fail(RESPIN_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  if (D < 128 || D > 65536 || D % 128)
+    return fail(RESPIN_ERR_UNSUPPORTED, "D=%d: need 128 <= D <= 65536 and D %% 128 == 0", D);
+  if (r < 1 || r > kPrR) return fail(RESPIN_ERR_UNSUPPORTED, "r=%d: subspace plans need 1 <= r <= %d", r, kPrR);
+  if (Q == nullptr || R_sub == nullptr) return fail(RESPIN_ERR_INVALID_ARG, "Q and R_sub must be non-NULL");
+  if (flags & ~(RESPIN_H_FP32_DEBUG | RESPIN_ACT_INT3))
+    return fail(RESPIN_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
+  if (fault_at("plan_alloc")) return fail(RESPIN_ERR_OOM, "injected fault at plan_alloc");
+  respin_plan_s* p = new respin_plan_s();
+  p->D = D; p->r = r; p->r_pad = kPrR; p->flags = flags; p->subspace = true;
+  cudaError_t e = cudaGetDevice(&p->device);
+  if (e != cudaSuccess) { delete p; return cuda_fail(e, "cudaGetDevice"); }
+  respin_status_t st = configure_pair(D, (flags & RESPIN_H_FP32_DEBUG) != 0, p);
+  if (st != RESPIN_OK) { delete p; return st; }
+  // Q as bf16 (round to nearest even), as the kernel's two fragment streams;
+  // M = R_sub - I formed exactly in double and rounded once to float, zero
+  // padded.
+  std::vector<uint16_t> qb(static_cast<size_t>(D) * r);
+  std::vector<uint32_t> qpk(static_cast<size_t>(D) * kPrR);   // 2 streams of D * 32 bf16
+  for (size_t i = 0; i < qb.size(); ++i) {
+    const __nv_bfloat16 v = __float2bfloat16_rn(Q[i]);
+    qb[i] = *reinterpret_cast<const uint16_t*>(&v);
+  }
+  pr_pack_frags(qb.data(), D, r, qpk.data(), qpk.data() + qpk.size() / 2);
+  std::vector<float> m(kPrR * kPrR, 0.0f);
+  for (int i = 0; i < r; ++i)
+    for (int j = 0; j < r; ++j)
+      m[i * kPrR + j] = static_cast<float>(static_cast<double>(R_sub[static_cast<size_t>(i) * r + j]) - (i == j ? 1.0 : 0.0));
+  e = cudaMalloc(&p->q_pair, qpk.size() * sizeof(uint32_t));
+  if (e == cudaSuccess) e = cudaMalloc(&p->m_pair, m.size() * sizeof(float));
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    if (p->q_pair) cudaFree(p->q_pair);
+    delete p;
+    return fail(RESPIN_ERR_OOM, "cudaMalloc subspace factors: %s", cudaGetErrorString(e));
+  }
+  e = cudaMemcpy(p->q_pair, qpk.data(), qpk.size() * sizeof(uint32_t), cudaMemcpyHostToDevice);
+  if (e == cudaSuccess) e = cudaMemcpy(p->m_pair, m.data(), m.size() * sizeof(float), cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) {
+    cudaFree(p->q_pair);
+    cudaFree(p->m_pair);
+    delete p;
+    return cuda_fail(e, "cudaMemcpy subspace factors");
+  }
+  {
+    std::lock_guard<std::mutex> lk(g_plans_mu);
+    g_plans.insert(p);
+  }
+  *out = p;
+  return ok();
+}
+
 respin_status_t respin_plan_destroy(respin_plan_t plan) {
   t_last_error.clear();
   if (plan == nullptr) return ok();
@@ -474,12 +561,14 @@ respin_status_t respin_plan_destroy(respin_plan_t plan) {
     if (!g_plans.erase(plan)) return fail(RESPIN_ERR_INVALID_ARG, "unknown or destroyed plan");
   }
   respin_status_t st = RESPIN_OK;
-  if (plan->factors) {
+  if (plan->factors || plan->q_pair) {
     int cur = -1;
     cudaGetDevice(&cur);
     cudaSetDevice(plan->device);
     cudaError_t e = cudaDeviceSynchronize();
-    if (e == cudaSuccess) e = cudaFree(plan->factors);
+    if (e == cudaSuccess && plan->factors) e = cudaFree(plan->factors);
+    if (e == cudaSuccess && plan->q_pair) e = cudaFree(plan->q_pair);
+    if (e == cudaSuccess && plan->m_pair) e = cudaFree(plan->m_pair);
     if (e == cudaSuccess && plan->factors_small) e = cudaFree(plan->factors_small);
     if (e == cudaSuccess && plan->factors_tiny) e = cudaFree(plan->factors_tiny);
     if (e != cudaSuccess) st = cuda_fail(e, "releasing plan factors");
@@ -525,6 +614,40 @@ respin_status_t respin_boundary_forward(respin_plan_t plan, const void* x, const
     }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "boundary_rowwise_kernel launch");
+    return ok();
+  }
+
+  if (plan->subspace) {
+    // T <= 8 tokens per tile so that every pair gets the same number of tiles
+    const long long per = static_cast<long long>(plan->pair_max) * kPrT;
+    const int k = static_cast<int>((N + per - 1) / per);
+    const long long slots = static_cast<long long>(plan->pair_max) * k;
+    int T = static_cast<int>((N + slots - 1) / slots);
+    if (T < 1) T = 1;
+    const int ntiles = (N + T - 1) / T;
+    const int pairs = ntiles < plan->pair_max ? ntiles : plan->pair_max;
+    CUtensorMap tmR, tmX;
+    if (!make_tmap_bf16_tile(&tmR, residual, N, D, kPrT) || !make_tmap_bf16_tile(&tmX, x, N, D, kPrT))
+      return fail(RESPIN_ERR_CUDA, "cuTensorMapEncodeTiled failed for the residual / x tiles");
+    const uint4* pf = reinterpret_cast<const uint4*>(plan->q_pair);
+    const uint4* rf = reinterpret_cast<const uint4*>(plan->q_pair + static_cast<size_t>(D) * kPrR / 2);
+    const float* mg = plan->m_pair;
+    int Dv = D;
+    void* args[] = {&tmR, &tmX, &pf, &rf, &mg, &N, &Dv, &T, &h_out, &q_packed, &scale, &qmax};
+    cudaLaunchConfig_t lc = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    lc.gridDim = dim3(static_cast<unsigned>(2 * pairs), 1, 1);
+    lc.blockDim = dim3(kPrThreads, 1, 1);
+    lc.dynamicSmemBytes = plan->pair_smem;
+    lc.stream = s;
+    lc.attrs = attr;
+    lc.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelExC(&lc, plan->pair_fn, args);
+    if (e != cudaSuccess) return cuda_fail(e, "boundary_pair_kernel launch");
     return ok();
   }
 
@@ -791,6 +914,26 @@ respin_status_t respin_selftest_wait_limit(unsigned limit_us, void* stream) {
   selftest_wait_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(static_cast<uint64_t>(limit_us) * 1000u);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "selftest_wait_kernel launch");
+  return ok();
+}
+
+respin_status_t respin_fuse_weight(int O, int K, const float* W, const float* R_in, const float* R_out,
+                                   float* W_fused) {
+  t_last_error.clear();
+  bool ok_ = false;
+  try {
+    ok_ = host::fuse_weight(O, K, W, R_in, R_out, W_fused);
+  } catch (const std::bad_alloc&) {
+    return fail(RESPIN_ERR_OOM, "host memory for the float64 copies of W and the rotations");
+  }
+  if (!ok_) return fail(RESPIN_ERR_INVALID_ARG, "need O > 0, K > 0 and non-NULL W, R_in, W_fused");
+  return ok();
+}
+
+respin_status_t respin_quantize_weight(int O, int K, const float* W, int qmax, uint8_t* q_w, float* scale_w) {
+  t_last_error.clear();
+  if (!host::quantize_weight_rows(O, K, W, qmax, q_w, scale_w))
+    return fail(RESPIN_ERR_INVALID_ARG, "need O > 0, even K > 0, qmax 7 or 3 and non-NULL pointers");
   return ok();
 }
 

@@ -121,3 +121,54 @@ def check_codes_end_to_end(q_packed, codes_ref):
     frac = float(np.mean(d != 0))
     assert frac <= CODE_MISMATCH_FRAC, f"code mismatch fraction {frac}"
     return frac
+
+
+def subspace_of(fx: W.BoundaryFixture):
+    """float32 (Q, R_sub) of the fixture's stored subspace form."""
+    Qr, R = W.subspace_factors(fx.Q, fx.theta, fx.r)
+    return Qr.astype(np.float32), R.astype(np.float32)
+
+
+def run_boundary_subspace(fx: W.BoundaryFixture, *, f32: bool, residual=True,
+                          h_out=True, device="cuda", qmax=7):
+    """respin_boundary_forward with a plan made by respin_plan_create_subspace
+    from the fixture's (Q, R_sub); returns numpy results."""
+    D, N, r = fx.D, fx.N, fx.r
+    flags = (rq.RESPIN_H_FP32_DEBUG if f32 else 0) | (rq.RESPIN_ACT_INT3 if qmax == 3 else 0)
+    Q32, R32 = subspace_of(fx)
+    plan = rq.SubspacePlan(D, r, Q32, R32, flags)
+    x = fx.x.to(device)
+    res = fx.residual.to(device) if residual else None
+    h = None
+    if h_out:
+        h = torch.empty(N, D, device=device, dtype=torch.float32 if f32 else torch.bfloat16)
+    q = torch.full((N, D // 2), 0xAB, device=device, dtype=torch.uint8)
+    s = torch.full((N,), -1.0, device=device, dtype=torch.float32)
+    rq.respin_boundary_forward(plan, x, res, h, q, s)
+    torch.cuda.synchronize()
+    assert rq.respin_device_status() == 0
+    plan.destroy()
+    out = dict(q=q.cpu().numpy(), scale=s.cpu().numpy())
+    if h is not None:
+        out["h"] = (h.cpu().numpy() if f32 else
+                    h.view(torch.int16).cpu().numpy().view(np.uint16))
+    return out
+
+
+def oracle_boundary_subspace(fx: W.BoundaryFixture, rows=None, residual=True, qmax=7):
+    """Oracle for a subspace plan of the fixture (optionally a row subset)."""
+    x = fx.x.float().numpy()
+    res = fx.residual.float().numpy() if residual else None
+    if rows is not None:
+        x = x[rows]
+        res = res[rows] if res is not None else None
+    Q32, R32 = subspace_of(fx)
+    return O.boundary_reference_subspace(x, res, Q32, R32, qmax)
+
+
+def subspace_corr_factors(fx: W.BoundaryFixture):
+    """(U, V) with (res U) V^T equal to the subspace plan's correction term
+    (U = bf16(Q), V = bf16(Q) M, float64)."""
+    Q32, R32 = subspace_of(fx)
+    Qq, M = O.subspace_plan_factors(Q32, R32)
+    return Qq, Qq @ M
