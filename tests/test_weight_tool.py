@@ -74,3 +74,26 @@ def test_weight_tool_validation():
     assert rq.lib.respin_quantize_weight(2, 3, p, 7, qb, p) == rq.RESPIN_ERR_INVALID_ARG   # odd K
     assert rq.lib.respin_quantize_weight(2, 4, p, 5, qb, p) == rq.RESPIN_ERR_INVALID_ARG   # qmax
     assert rq.last_error()
+
+
+def test_fuse_weight_permutation_permutes_columns():
+    """A permutation as the input rotation only reorders W's columns."""
+    rs = np.random.default_rng(9)
+    W = rs.standard_normal((16, 64)).astype(np.float32)
+    perm = rs.permutation(64)
+    P = np.zeros((64, 64), np.float32)
+    P[perm, np.arange(64)] = 1.0          # (W P)[:, j] = W[:, perm[j]]
+    got = rq.respin_fuse_weight(W, P)
+    assert np.array_equal(got, W[:, perm])
+
+
+@pytest.mark.parametrize("qmax,bytes_", [(7, [0xC7, 0x02]), (3, [0xE3, 0x01])])
+def test_quantize_weight_hand_worked_row(qmax, bytes_):
+    """Row [2, -1, 0.5, 0]: inv = qmax/2; -1*inv = -qmax/2 is a tie that goes
+    to the even integer (-4 for INT4, -2 for INT3); scale = 2/qmax."""
+    W = np.array([[2.0, -1.0, 0.5, 0.0]], np.float32)
+    q, sc = rq.respin_quantize_weight(W, qmax)
+    assert list(q[0]) == bytes_
+    assert sc[0] == np.float32(2.0) / np.float32(qmax)
+    qo, so = O.quantize_weight_rows(W, qmax)
+    assert list(qo[0]) == bytes_ and so[0] == sc[0]
