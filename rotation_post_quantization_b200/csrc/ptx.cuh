@@ -197,6 +197,13 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, int 
       : "memory");
 }
 
+// Prefetch of one 2-D tensor-map box into L2 (no shared memory, no
+// completion to wait for); same coordinate rule as tma_load_2d.
+__device__ __forceinline__ void tma_prefetch_2d(const void* tmap, int x, int y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(tmap), "r"(x), "r"(y)
+               : "memory");
+}
+
 // 2-D tensor copy shared -> global through a tensor map (bulk-group
 // completion). Elements outside the tensor are not written.
 __device__ __forceinline__ void tma_store_2d(const void* tmap, int x, int y, uint32_t src) {

@@ -618,11 +618,18 @@ respin_status_t respin_boundary_forward(respin_plan_t plan, const void* x, const
   }
 
   if (plan->subspace) {
-    // T <= 8 tokens per tile so that every pair gets the same number of tiles
-    const long long per = static_cast<long long>(plan->pair_max) * kPrT;
-    const int k = static_cast<int>((N + per - 1) / per);
-    const long long slots = static_cast<long long>(plan->pair_max) * k;
-    int T = static_cast<int>((N + slots - 1) / slots);
+    // T <= 16 tokens per tile. While full tiles need at most half of the
+    // co-resident pairs (one CTA per SM), tiles are full; beyond that T is
+    // chosen so that every pair gets the same number of tiles (two CTAs per
+    // SM share the work evenly).
+    const long long tiles16 = (static_cast<long long>(N) + kPrT - 1) / kPrT;
+    int T = kPrT;
+    if (tiles16 > plan->pair_max / 2) {
+      const long long per = static_cast<long long>(plan->pair_max) * kPrT;
+      const int k = static_cast<int>((N + per - 1) / per);
+      const long long slots = static_cast<long long>(plan->pair_max) * k;
+      T = static_cast<int>((N + slots - 1) / slots);
+    }
     if (T < 1) T = 1;
     const int ntiles = (N + T - 1) / T;
     const int pairs = ntiles < plan->pair_max ? ntiles : plan->pair_max;
