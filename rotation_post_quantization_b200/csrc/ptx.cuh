@@ -25,6 +25,9 @@ enum StatusSite : int {
   kSiteGemmPackedEmpty = 205,// GEMM TMA warp: waiting for a free packed stage
   kSitePairPeer = 301,       // pair boundary kernel: waiting for the peer CTA's partials
   kSitePairLoad = 302,       // pair boundary kernel: waiting for a staged block or the basis
+  kSiteTcLoad = 401,         // tensor-core boundary passes: waiting for a staged tile
+  kSiteTcFree = 402,         // tensor-core boundary passes: waiting for a free stage
+  kSiteTcAccum = 403,        // tensor-core boundary passes: waiting for accumulators / operand A
   kSiteSelfTest = 901,       // respin_selftest_wait_limit: a wait that nothing completes
 };
 
@@ -413,6 +416,18 @@ __device__ __forceinline__ void tc_mma_i8(uint32_t d_tmem, uint64_t adesc, uint6
       : "memory");
 }
 
+// One 128 x N x 16 bf16 MMA with fp32 accumulation: D[tmem] (+)= A * B^T,
+// both operands K-major in shared memory.
+__device__ __forceinline__ void tc_mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrive on `bar` once all tcgen05 operations issued so far by this thread
 // have completed.
 __device__ __forceinline__ void tc_commit(uint32_t bar) {
@@ -460,6 +475,16 @@ __host__ __device__ constexpr uint32_t umma_idesc_s8(int M, int N) {
   return (2u << 4)                                   // D format: S32
          | (1u << 7)                                 // A: signed 8-bit
          | (1u << 10)                                // B: signed 8-bit
+         | (static_cast<uint32_t>(N >> 3) << 17)     // N / 8
+         | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
+}
+
+// Instruction descriptor: kind::f16 with bf16 A and B, fp32 accumulator,
+// both operands K-major, shape M x N.
+__host__ __device__ constexpr uint32_t umma_idesc_bf16(int M, int N) {
+  return (1u << 4)                                   // D format: F32
+         | (1u << 7)                                 // A: BF16
+         | (1u << 10)                                // B: BF16
          | (static_cast<uint32_t>(N >> 3) << 17)     // N / 8
          | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
 }

@@ -22,6 +22,7 @@
 #include "boundary_kernels.cuh"
 #include "boundary_pair.cuh"
 #include "boundary_rowtile.cuh"
+#include "boundary_tc.cuh"
 #include "factor_builder.h"
 #include "weight_tool.h"
 #include "w4a4_gemm_kernels.cuh"
@@ -103,7 +104,20 @@ struct respin_plan_s {
   const void* pair_fn = nullptr;
   size_t pair_smem = 0;
   int pair_max = 0;              // co-resident CTA pairs
+  // Tensor-core passes for padded ranks 64 / 128 (boundary_tc.cuh): tensor
+  // maps of the plan's U^T [r_pad, D] and V [D, r_pad] (the factor layout of
+  // the shared-memory cluster kernel).
+  bool has_tc = false;
+  CUtensorMap tm_ut, tm_v;
+  const void* tc_proj_fn = nullptr;
+  const void* tc_re_fn = nullptr;
+  size_t tc_proj_smem = 0, tc_re_smem = 0;
+  int sms = 0;
 };
+
+// Calls with at least this many tokens take the tensor-core passes when the
+// plan has them (padded rank 64 or 128).
+constexpr int kTcMinTokens = 256;
 
 // Calls with at most this many tokens use cfg_small when the plan has one
 // (row tiles: one 16-token tile per SM; a 4-CTA cluster tile chain is about a
@@ -160,6 +174,64 @@ bool make_tmap_bf16_tile(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 2-D bf16 tensor map over a row-major [rows, cols] array with a
+// {box_cols, box_rows} box and the given swizzle.
+bool make_tmap_bf16(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_cols,
+                    uint32_t box_rows, CUtensorMapSwizzle swz) {
+  EncodeTiledFn fn = encode_tiled();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * 2};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int RP>
+const void* tc_proj_fn() {
+  return reinterpret_cast<const void*>(&boundary_tc_project_kernel<RP>);
+}
+template <int RP, bool F32>
+const void* tc_re_fn() {
+  return reinterpret_cast<const void*>(&boundary_tc_reproject_kernel<RP, F32>);
+}
+
+// The tensor-core passes of a plan whose factors are stored as U^T then V
+// (padded rank 64 or 128). Leaves has_tc false where they do not apply.
+void configure_tc(respin_plan_s* p) {
+  const int D = p->D, RP = p->r_pad;
+  if ((RP != 64 && RP != 128) || p->cfg.kind != kClusterSmem || p->cfg.rf || p->factors == nullptr) return;
+  const bool f32 = (p->flags & RESPIN_H_FP32_DEBUG) != 0;
+  const void* pf = RP == 64 ? tc_proj_fn<64>() : tc_proj_fn<128>();
+  const void* rf = RP == 64 ? (f32 ? tc_re_fn<64, true>() : tc_re_fn<64, false>())
+                            : (f32 ? tc_re_fn<128, true>() : tc_re_fn<128, false>());
+  const size_t ps = RP == 64 ? TcProjCfg<64>::kSmem : TcProjCfg<128>::kSmem;
+  const size_t rs = RP == 64 ? TcReCfg<64>::kSmem : TcReCfg<128>::kSmem;
+  if (cudaFuncSetAttribute(pf, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(ps)) != cudaSuccess ||
+      cudaFuncSetAttribute(rf, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(rs)) != cudaSuccess) {
+    cudaGetLastError();
+    return;
+  }
+  const __nv_bfloat16* ut = p->factors;
+  const __nv_bfloat16* v = p->factors + static_cast<size_t>(RP) * D;
+  if (!make_tmap_bf16(&p->tm_ut, ut, RP, D, 64, RP, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tmap_bf16(&p->tm_v, v, D, RP, 64, kTcBN, CU_TENSOR_MAP_SWIZZLE_128B))
+    return;
+  int sms = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, p->device) != cudaSuccess || sms <= 0) {
+    cudaGetLastError();
+    return;
+  }
+  p->tc_proj_fn = pf;
+  p->tc_re_fn = rf;
+  p->tc_proj_smem = ps;
+  p->tc_re_smem = rs;
+  p->sms = sms;
+  p->has_tc = true;
 }
 
 template <int R, int W, int NB, bool F32>
@@ -488,7 +560,7 @@ respin_status_t respin_plan_create(respin_plan_t* out, int D, int r, const float
       return st2 != RESPIN_OK ? st2 : fail(RESPIN_ERR_OOM, "factor upload failed");
     }
   }
-  // The row kernels need the shared-memory carve-out only for their reduction.
+  if (r > 0) configure_tc(p);
   {
     std::lock_guard<std::mutex> lk(g_plans_mu);
     g_plans.insert(p);
@@ -655,6 +727,51 @@ respin_status_t respin_boundary_forward(respin_plan_t plan, const void* x, const
     lc.numAttrs = 1;
     cudaError_t e = cudaLaunchKernelExC(&lc, plan->pair_fn, args);
     if (e != cudaSuccess) return cuda_fail(e, "boundary_pair_kernel launch");
+    return ok();
+  }
+
+  if (plan->has_tc && N >= kTcMinTokens && h_out != nullptr) {
+    // Three launches: y partials (into the code buffer's rows), h' with the
+    // per-token amax (into the scale buffer), codes and scales.
+    const int RP = plan->r_pad;
+    int KB = D / 64;
+    const int mtiles = (N + kTcBM - 1) / kTcBM;
+    int S = (plan->sms + mtiles - 1) / mtiles;
+    const int smax = D / (8 * RP);   // partials of a token fit in its D / 2 code bytes
+    if (S > smax) S = smax;
+    if (S > KB) S = KB;
+    if (S > 8) S = 8;
+    if (S < 1) S = 1;
+    CUtensorMap tmR, tmRc, tmXc;
+    if (!make_tmap_bf16(&tmR, residual, N, D, 64, kTcBM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_tmap_bf16(&tmRc, residual, N, D, kTcChunk, kTcBM, CU_TENSOR_MAP_SWIZZLE_64B) ||
+        !make_tmap_bf16(&tmXc, x, N, D, kTcChunk, kTcBM, CU_TENSOR_MAP_SWIZZLE_64B))
+      return fail(RESPIN_ERR_CUDA, "cuTensorMapEncodeTiled failed for the tensor-core boundary tiles");
+    cudaError_t e = cudaMemsetAsync(scale, 0, static_cast<size_t>(N) * sizeof(float), s);
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the scale buffer");
+    uint8_t* ypart = static_cast<uint8_t*>(q_packed);
+    int ypitch = D / 2, Nv = N, Dv = D;
+    {
+      void* args[] = {&tmR, &plan->tm_ut, &Nv, &KB, &S, &ypart, &ypitch};
+      e = cudaLaunchKernel(plan->tc_proj_fn, dim3(static_cast<unsigned>(mtiles * S)), dim3(128), args,
+                           plan->tc_proj_smem, s);
+      if (e != cudaSuccess) return cuda_fail(e, "boundary_tc_project_kernel launch");
+    }
+    {
+      const long long tiles = static_cast<long long>(mtiles) * (D / kTcBN);
+      const int grid = tiles < plan->sms ? static_cast<int>(tiles) : plan->sms;
+      const uint8_t* yp = ypart;
+      void* args[] = {&tmRc, &tmXc, &plan->tm_v, &Nv, &Dv, &S, &yp, &ypitch, &h_out, &scale};
+      e = cudaLaunchKernel(plan->tc_re_fn, dim3(static_cast<unsigned>(grid)), dim3(192), args, plan->tc_re_smem, s);
+      if (e != cudaSuccess) return cuda_fail(e, "boundary_tc_reproject_kernel launch");
+    }
+    {
+      const int grid = N < plan->sms * 8 ? N : plan->sms * 8;
+      if (f32) boundary_quant_rows_kernel<true><<<grid, 256, 0, s>>>(h_out, N, D, q_packed, scale, qmax);
+      else boundary_quant_rows_kernel<false><<<grid, 256, 0, s>>>(h_out, N, D, q_packed, scale, qmax);
+      e = cudaGetLastError();
+      if (e != cudaSuccess) return cuda_fail(e, "boundary_quant_rows_kernel launch");
+    }
     return ok();
   }
 

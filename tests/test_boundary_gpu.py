@@ -36,6 +36,12 @@ CASES = [
     ("rowtile_d4096_ragged", 4096, 1301, 32, 64, 0.1, 8, 50.0, "normal"),
     ("rowtile_d4096_nu1", 4096, 1296, 32, 64, 1.0, 8, 50.0, "normal"),
     ("rowtile_d2048_r16", 2048, 1290, 16, 32, 0.5, 4, 20.0, "student_t3"),
+    # at least 256 tokens with padded rank 64 / 128: the tensor-core passes
+    # (ragged token tiles, several K splits, one K split at D = 1024)
+    ("tc_d8192_r64", 8192, 300, 64, 128, 0.1, 16, 100.0, "student_t3"),
+    ("tc_d8192_r128", 8192, 333, 128, 128, 0.1, 16, 100.0, "student_t3"),
+    ("tc_d4096_r48", 4096, 520, 48, 64, 0.1, 8, 50.0, "normal"),
+    ("tc_d1024_r128", 1024, 700, 128, 128, 0.5, 4, 50.0, "normal"),
 ]
 
 
@@ -219,6 +225,8 @@ def test_rank_sweep_eckart_young_70b():
         got = run_boundary(fx, f32=True)
         x = fx.x.float().numpy().astype(np.float64)
         res = fx.residual.float().numpy().astype(np.float64)
+        # the kernel's correction against its own (plan-rounded) rank-r factors
+        check_corr(got["h"], x, res, *O.plan_factors(fx.U.astype(np.float32), fx.V.astype(np.float32)))
         hd = O.boundary_fp64(x, res, Uk, Vk)
         e = np.linalg.norm(got["h"].astype(np.float64) - hd, axis=1)
         rn = np.linalg.norm(res, axis=1)
