@@ -819,27 +819,37 @@ boundary_cluster_smem_kernel(const bf16* __restrict__ x, const bf16* __restrict_
 }
 
 // One CTA per token row (grid-stride): r == 0 or no residual. h = residual + x.
-template <int THREADS, bool F32OUT>
+// VPT: 16-byte vectors per thread (D <= THREADS * 8 * VPT); the host picks
+// the smallest that covers D, so registers (and the CTAs an SM holds) follow
+// the row length.
+template <int THREADS, int VPT, bool F32OUT>
 __global__ void __launch_bounds__(THREADS)
 boundary_rowwise_kernel(const bf16* __restrict__ x, const bf16* __restrict__ res, int N, int D,
                         void* __restrict__ h_out, uint8_t* __restrict__ q_out,
                         float* __restrict__ scale_out, float qmax) {
-  constexpr int VPT = 8;  // 16-byte vectors per thread (D <= THREADS * 64)
   __shared__ float red[THREADS / 32];
   __shared__ float s_inv;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nv = D / 8;
   for (int row = blockIdx.x; row < N; row += gridDim.x) {
     const size_t base = static_cast<size_t>(row) * D;
-    uint4 hv[VPT];
+    uint4 hv[VPT], xin[VPT], rin[VPT];
     float amax = 0.f;
+    // all loads of the row first (predicated, so they are in flight together)
+#pragma unroll
+    for (int j = 0; j < VPT; ++j) {
+      const int v = tid + j * THREADS;
+      xin[j] = rin[j] = make_uint4(0u, 0u, 0u, 0u);
+      if (v < nv) {
+        xin[j] = __ldg(reinterpret_cast<const uint4*>(x + base) + v);
+        if (res != nullptr) rin[j] = __ldg(reinterpret_cast<const uint4*>(res + base) + v);
+      }
+    }
 #pragma unroll
     for (int j = 0; j < VPT; ++j) {
       const int v = tid + j * THREADS;
       if (v >= nv) break;
-      const uint4 xv = __ldg(reinterpret_cast<const uint4*>(x + base) + v);
-      uint4 rv = make_uint4(0u, 0u, 0u, 0u);
-      if (res != nullptr) rv = __ldg(reinterpret_cast<const uint4*>(res + base) + v);
+      const uint4 xv = xin[j], rv = rin[j];
       const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
       const uint32_t rw[4] = {rv.x, rv.y, rv.z, rv.w};
       uint32_t hw[4];

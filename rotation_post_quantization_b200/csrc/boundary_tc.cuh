@@ -56,7 +56,7 @@ __device__ __forceinline__ uint32_t tc_sw64(int r, int j) {
 template <int RP>
 struct TcProjCfg {
   static_assert(RP == 64 || RP == 128, "padded rank");
-  static constexpr int STG = 6;                       // K-block stages
+  static constexpr int STG = RP == 64 ? 8 : 6;        // K-block stages (192 KB either way)
   static constexpr uint32_t ABytes = kTcKBlock;       // 128 tokens x 64
   static constexpr uint32_t BBytes = RP * 128;        // RP rows of U^T x 64
   static constexpr uint32_t Stage = ABytes + BBytes;
@@ -173,6 +173,7 @@ struct TcReCfg {
   static constexpr int BST = 2;                                // V tile stages
   static constexpr uint32_t BBytes = KBR * kTcBN * 128;        // 128 rows of V x RP
   static constexpr int CST = RP == 128 ? 6 : 8;                // residual + x chunk stages
+  static constexpr int HST = CST / 2;                          // stages of each half's ring
   static constexpr uint32_t CHalf = kTcBM * kTcChunk * 2;      // 128 rows x 32 columns bf16 (8 KB)
   static constexpr uint32_t CBytes = 2 * CHalf;                // residual then x
   static constexpr uint32_t oA = 0;
@@ -183,7 +184,7 @@ struct TcReCfg {
   static constexpr int kBars = 2 * BST + 2 * CST + 4 + 3;
   static constexpr uint32_t oMisc = oBars + kBars * 8;        // tmem slot, abort flag
   static constexpr uint32_t kSmem = oMisc + 16 + 1024;
-  static constexpr int kThreads = 192;                         // producer, MMA, 4 epilogue warps
+  static constexpr int kThreads = 320;                         // producer, MMA, 8 epilogue warps
   static_assert(kSmem <= 227 * 1024, "shared memory");
 };
 
@@ -193,7 +194,7 @@ struct TcReCfg {
 // [b T / G, (b+1) T / G). amax: the scale buffer, zero on entry, receives
 // the bit pattern of max |h'| per token.
 template <int RP, bool F32OUT>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
 boundary_tc_reproject_kernel(const __grid_constant__ CUtensorMap tmRc, const __grid_constant__ CUtensorMap tmXc,
                              const __grid_constant__ CUtensorMap tmV, int N, int D, int S,
                              const uint8_t* __restrict__ ypart, int ypitch, void* __restrict__ h_out,
@@ -227,8 +228,8 @@ boundary_tc_reproject_kernel(const __grid_constant__ CUtensorMap tmRc, const __g
   if (tid == 0) {
     for (int s = 0; s < C::BST; ++s) { mbar_init(bfull(s), 1); mbar_init(bempty(s), 1); }
     for (int s = 0; s < C::CST; ++s) { mbar_init(cfull(s), 1); mbar_init(cempty(s), 4); }
-    for (int a = 0; a < 2; ++a) { mbar_init(afull(a), 1); mbar_init(aempty(a), 4); }
-    mbar_init(opa_full, 4);
+    for (int a = 0; a < 2; ++a) { mbar_init(afull(a), 1); mbar_init(aempty(a), 8); }
+    mbar_init(opa_full, 8);
     mbar_init(opa_empty, 1);
     mbar_init(fin, 1);
     *abort_flag = 0;
@@ -248,15 +249,20 @@ boundary_tc_reproject_kernel(const __grid_constant__ CUtensorMap tmRc, const __g
 
   if (warp == 0) {
     // ---- producer lanes: lane c < CST owns chunk stage c, lane 16 + s owns
-    // V stage s; each stage has at most one copy in flight.
+    // V stage s; each stage has at most one copy in flight. The chunk stages
+    // form two rings, one per epilogue half (stages h HST .. h HST + HST - 1
+    // carry half h's chunks 2h, 2h + 1 of every tile, in order), so every
+    // stage is consumed by the same four warps in order and no consumer can
+    // run two phases ahead of a stage.
     int last = -1;   // this lane's last issued use (for the final drain)
     if (lane < C::CST) {
-      const int nq = 4 * nloc;
-      for (int q = lane; q < nq; q += C::CST) {
+      const int h = lane / C::HST, j = lane % C::HST;
+      const int np = 2 * nloc;   // chunks of half h
+      for (int pidx = j; pidx < np; pidx += C::HST) {
         if (*abort_flag) break;
-        const int u = q / C::CST;
+        const int u = pidx / C::HST;
         if (!mbar_wait(cempty(lane), (u & 1) ^ 1, kSiteTcFree)) { *abort_flag = 1; break; }
-        const int i = q >> 2, c = q & 3;
+        const int i = pidx >> 1, c = 2 * h + (pidx & 1);
         const int x0 = tile_n(i) * kTcBN + c * kTcChunk, y0 = tile_m(i) * kTcBM;
         const uint32_t dst = base + C::oC + lane * C::CBytes;
         mbar_arrive_expect_tx(cfull(lane), C::CBytes);
@@ -311,9 +317,11 @@ boundary_tc_reproject_kernel(const __grid_constant__ CUtensorMap tmRc, const __g
     }
     if (lane == 0) tc_commit(fin);   // completes once every issued MMA has
   } else {
-    // ---- epilogue warps: TMEM lane quarter qd = warp % 4 holds tile rows
-    // 32 qd .. 32 qd + 31; thread = one token row.
+    // ---- epilogue warps 2..9: TMEM lane quarter qd = warp % 4 holds tile
+    // rows 32 qd .. 32 qd + 31 (thread = one token row); warps 2-5 take the
+    // 32-column chunks 0 and 1 of a tile, warps 6-9 chunks 2 and 3.
     const int qd = warp & 3;
+    const int half = (warp - 2) >> 2;
     const int r = 32 * qd + lane;
     int seg = 0;
     bool ok = true;
@@ -330,7 +338,7 @@ boundary_tc_reproject_kernel(const __grid_constant__ CUtensorMap tmRc, const __g
         uint8_t* arow = smem + C::oA + (r >> 3) * 1024 + (r & 7) * 128;
         const float* yp = reinterpret_cast<const float*>(ypart + static_cast<size_t>(tok < N ? tok : 0) * ypitch);
 #pragma unroll 1
-        for (int c8 = 0; c8 < RP / 8; ++c8) {
+        for (int c8 = half * (RP / 16); c8 < (half + 1) * (RP / 16); ++c8) {
           float y[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) y[e] = 0.f;
@@ -361,12 +369,13 @@ boundary_tc_reproject_kernel(const __grid_constant__ CUtensorMap tmRc, const __g
       tc_fence_after();
       float rmax = 0.f;
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        const int q = 4 * i + c, cs = q % C::CST;
+      for (int c = 2 * half; c < 2 * half + 2; ++c) {
+        const int pidx = 2 * i + (c - 2 * half);   // position in this half's chunk ring
+        const int cs = half * C::HST + pidx % C::HST;
         uint32_t v[32];
         tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(32 * qd) << 16) + ab * kTcBN + kTcChunk * c, v);
         tmem_wait_ld();
-        if (ok) ok = mbar_wait(cfull(cs), (q / C::CST) & 1, kSiteTcLoad);
+        if (ok) ok = mbar_wait(cfull(cs), (pidx / C::HST) & 1, kSiteTcLoad);
         ok = __all_sync(0xffffffffu, ok);
         const uint8_t* rs = smem + C::oC + cs * C::CBytes;
         const uint8_t* xs = rs + C::CHalf;
@@ -435,22 +444,37 @@ template <bool F32IN>
 __global__ void __launch_bounds__(256)
 boundary_quant_rows_kernel(const void* __restrict__ h, int N, int D, uint8_t* __restrict__ q_out,
                            float* __restrict__ scale_io, float qmax) {
+  constexpr int VPT = 8;   // 16-byte vectors of h' per thread per pass (D <= 16384 in one pass)
   const int tid = threadIdx.x;
   const int nv = D / 8;
   for (int row = blockIdx.x; row < N; row += gridDim.x) {
     const float amax = scale_io[row];
     float inv, sc;
     inv_and_scale(amax, qmax, inv, sc);
-    for (int v = tid; v < nv; v += 256) {
-      uint4 hv;
-      if constexpr (F32IN) {
-        const float4* hp = reinterpret_cast<const float4*>(static_cast<const float*>(h) + static_cast<size_t>(row) * D) + 2 * v;
-        const float4 a = hp[0], b = hp[1];
-        hv = make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y), pack_bf16x2(b.z, b.w));
-      } else {
-        hv = reinterpret_cast<const uint4*>(static_cast<const bf16*>(h) + static_cast<size_t>(row) * D)[v];
+    for (int v0 = 0; v0 < nv; v0 += 256 * VPT) {
+      uint4 hv[VPT];
+      // all loads first (predicated, in flight together), then the codes
+#pragma unroll
+      for (int j = 0; j < VPT; ++j) {
+        const int v = v0 + tid + 256 * j;
+        hv[j] = make_uint4(0u, 0u, 0u, 0u);
+        if (v < nv) {
+          if constexpr (F32IN) {
+            const float4* hp =
+                reinterpret_cast<const float4*>(static_cast<const float*>(h) + static_cast<size_t>(row) * D) + 2 * v;
+            const float4 a = hp[0], b = hp[1];
+            hv[j] = make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y),
+                               pack_bf16x2(b.z, b.w));
+          } else {
+            hv[j] = reinterpret_cast<const uint4*>(static_cast<const bf16*>(h) + static_cast<size_t>(row) * D)[v];
+          }
+        }
       }
-      reinterpret_cast<uint32_t*>(q_out + static_cast<size_t>(row) * (D / 2))[v] = quantize8(hv, inv);
+#pragma unroll
+      for (int j = 0; j < VPT; ++j) {
+        const int v = v0 + tid + 256 * j;
+        if (v < nv) reinterpret_cast<uint32_t*>(q_out + static_cast<size_t>(row) * (D / 2))[v] = quantize8(hv[j], inv);
+      }
     }
     __syncthreads();   // every thread has read amax before it is replaced
     if (tid == 0) scale_io[row] = sc;

@@ -108,6 +108,9 @@ struct respin_plan_s {
   // maps of the plan's U^T [r_pad, D] and V [D, r_pad] (the factor layout of
   // the shared-memory cluster kernel).
   bool has_tc = false;
+  int tc_rp = 0;                          // padded rank of the passes (64 or 128)
+  int tc_min_tokens = 0;                  // calls from this many tokens on take them
+  __nv_bfloat16* tc_factors = nullptr;    // own U^T / V copy when the plan's layout differs
   CUtensorMap tm_ut, tm_v;
   const void* tc_proj_fn = nullptr;
   const void* tc_re_fn = nullptr;
@@ -116,8 +119,16 @@ struct respin_plan_s {
 };
 
 // Calls with at least this many tokens take the tensor-core passes when the
-// plan has them (padded rank 64 or 128).
-constexpr int kTcMinTokens = 256;
+// plan has them: padded rank 64 / 128, and padded rank 16 / 32 on the
+// register-factor cluster kernel (D = 8192). Measured on B200 at D = 8192
+// (passes vs cluster kernel): r = 64: 33 vs 34 us at 256 tokens, 159 vs
+// 672 us at 8192; r = 32: 68 vs 62 us at 2048 tokens, 159 vs 222 us at 8192.
+#ifndef RESPIN_TC_MIN_TOKENS
+#define RESPIN_TC_MIN_TOKENS 256
+#endif
+#ifndef RESPIN_TC_MIN_TOKENS_LOW_RANK
+#define RESPIN_TC_MIN_TOKENS_LOW_RANK 4096
+#endif
 
 // Calls with at most this many tokens use cfg_small when the plan has one
 // (row tiles: one 16-token tile per SM; a 4-CTA cluster tile chain is about a
@@ -200,11 +211,18 @@ const void* tc_re_fn() {
   return reinterpret_cast<const void*>(&boundary_tc_reproject_kernel<RP, F32>);
 }
 
-// The tensor-core passes of a plan whose factors are stored as U^T then V
-// (padded rank 64 or 128). Leaves has_tc false where they do not apply.
-void configure_tc(respin_plan_s* p) {
-  const int D = p->D, RP = p->r_pad;
-  if ((RP != 64 && RP != 128) || p->cfg.kind != kClusterSmem || p->cfg.rf || p->factors == nullptr) return;
+// The tensor-core passes of a plan: padded rank 64 / 128 (factors already
+// stored as U^T then V), or padded rank 16 / 32 on the register-factor
+// cluster kernel (D = 8192 and other widths the row-tile kernel does not
+// take), which gets its own U^T / V copy padded to 64. ub / vb: the bf16 bits
+// of U and V, [D][r_pad]. Leaves has_tc false where the passes do not apply.
+void configure_tc(respin_plan_s* p, const uint16_t* ub, const uint16_t* vb) {
+  const int D = p->D;
+  const bool own = p->r_pad <= 32 && p->cfg.kind == kClusterRf;
+  if (!own && ((p->r_pad != 64 && p->r_pad != 128) || p->cfg.kind != kClusterSmem || p->cfg.rf ||
+               p->factors == nullptr))
+    return;
+  const int RP = own ? 64 : p->r_pad;
   const bool f32 = (p->flags & RESPIN_H_FP32_DEBUG) != 0;
   const void* pf = RP == 64 ? tc_proj_fn<64>() : tc_proj_fn<128>();
   const void* rf = RP == 64 ? (f32 ? tc_re_fn<64, true>() : tc_re_fn<64, false>())
@@ -216,8 +234,27 @@ void configure_tc(respin_plan_s* p) {
     cudaGetLastError();
     return;
   }
-  const __nv_bfloat16* ut = p->factors;
-  const __nv_bfloat16* v = p->factors + static_cast<size_t>(RP) * D;
+  if (own) {
+    std::vector<uint16_t> w(static_cast<size_t>(2) * D * RP, 0);   // U^T [RP][D] then V [D][RP]
+    for (int d = 0; d < D; ++d)
+      for (int j = 0; j < p->r_pad; ++j) {
+        w[static_cast<size_t>(j) * D + d] = ub[static_cast<size_t>(d) * p->r_pad + j];
+        w[static_cast<size_t>(RP) * D + static_cast<size_t>(d) * RP + j] = vb[static_cast<size_t>(d) * p->r_pad + j];
+      }
+    if (cudaMalloc(&p->tc_factors, w.size() * sizeof(uint16_t)) != cudaSuccess) {
+      cudaGetLastError();
+      p->tc_factors = nullptr;
+      return;
+    }
+    if (cudaMemcpy(p->tc_factors, w.data(), w.size() * sizeof(uint16_t), cudaMemcpyHostToDevice) != cudaSuccess) {
+      cudaGetLastError();
+      cudaFree(p->tc_factors);
+      p->tc_factors = nullptr;
+      return;
+    }
+  }
+  const __nv_bfloat16* ut = own ? p->tc_factors : p->factors;
+  const __nv_bfloat16* v = ut + static_cast<size_t>(RP) * D;
   if (!make_tmap_bf16(&p->tm_ut, ut, RP, D, 64, RP, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_tmap_bf16(&p->tm_v, v, D, RP, 64, kTcBN, CU_TENSOR_MAP_SWIZZLE_128B))
     return;
@@ -231,6 +268,8 @@ void configure_tc(respin_plan_s* p) {
   p->tc_proj_smem = ps;
   p->tc_re_smem = rs;
   p->sms = sms;
+  p->tc_rp = RP;
+  p->tc_min_tokens = own ? RESPIN_TC_MIN_TOKENS_LOW_RANK : RESPIN_TC_MIN_TOKENS;
   p->has_tc = true;
 }
 
@@ -559,8 +598,9 @@ respin_status_t respin_plan_create(respin_plan_t* out, int D, int r, const float
       delete p;
       return st2 != RESPIN_OK ? st2 : fail(RESPIN_ERR_OOM, "factor upload failed");
     }
+    configure_tc(p, ub.data(), vb.data());
+    t_last_error.clear();
   }
-  if (r > 0) configure_tc(p);
   {
     std::lock_guard<std::mutex> lk(g_plans_mu);
     g_plans.insert(p);
@@ -643,6 +683,7 @@ respin_status_t respin_plan_destroy(respin_plan_t plan) {
     if (e == cudaSuccess && plan->m_pair) e = cudaFree(plan->m_pair);
     if (e == cudaSuccess && plan->factors_small) e = cudaFree(plan->factors_small);
     if (e == cudaSuccess && plan->factors_tiny) e = cudaFree(plan->factors_tiny);
+    if (e == cudaSuccess && plan->tc_factors) e = cudaFree(plan->tc_factors);
     if (e != cudaSuccess) st = cuda_fail(e, "releasing plan factors");
     cudaSetDevice(cur);
   }
@@ -677,13 +718,16 @@ respin_status_t respin_boundary_forward(respin_plan_t plan, const void* x, const
     int sms = 148;
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, plan->device);
     const int grid = N < sms * 16 ? N : sms * 16;
-    if (D <= 256 * 64) {
-      if (f32) boundary_rowwise_kernel<256, true><<<grid, 256, 0, s>>>(xb, rb, N, D, h_out, q_packed, scale, qmax);
-      else boundary_rowwise_kernel<256, false><<<grid, 256, 0, s>>>(xb, rb, N, D, h_out, q_packed, scale, qmax);
-    } else {
-      if (f32) boundary_rowwise_kernel<1024, true><<<grid, 1024, 0, s>>>(xb, rb, N, D, h_out, q_packed, scale, qmax);
-      else boundary_rowwise_kernel<1024, false><<<grid, 1024, 0, s>>>(xb, rb, N, D, h_out, q_packed, scale, qmax);
-    }
+#define RESPIN_ROWWISE(TH, VP)                                                                           \
+  {                                                                                                     \
+    if (f32) boundary_rowwise_kernel<TH, VP, true><<<grid, TH, 0, s>>>(xb, rb, N, D, h_out, q_packed, scale, qmax); \
+    else boundary_rowwise_kernel<TH, VP, false><<<grid, TH, 0, s>>>(xb, rb, N, D, h_out, q_packed, scale, qmax);   \
+  }
+    if (D <= 256 * 8 * 2) RESPIN_ROWWISE(256, 2)
+    else if (D <= 256 * 8 * 4) RESPIN_ROWWISE(256, 4)
+    else if (D <= 256 * 8 * 8) RESPIN_ROWWISE(256, 8)
+    else RESPIN_ROWWISE(1024, 8)
+#undef RESPIN_ROWWISE
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "boundary_rowwise_kernel launch");
     return ok();
@@ -730,13 +774,13 @@ respin_status_t respin_boundary_forward(respin_plan_t plan, const void* x, const
     return ok();
   }
 
-  if (plan->has_tc && N >= kTcMinTokens && h_out != nullptr) {
+  if (plan->has_tc && N >= plan->tc_min_tokens && h_out != nullptr) {
     // Three launches: y partials (into the code buffer's rows), h' with the
     // per-token amax (into the scale buffer), codes and scales.
-    const int RP = plan->r_pad;
+    const int RP = plan->tc_rp;
     int KB = D / 64;
     const int mtiles = (N + kTcBM - 1) / kTcBM;
-    int S = (plan->sms + mtiles - 1) / mtiles;
+    int S = plan->sms / mtiles;   // one CTA per SM, all in one wave
     const int smax = D / (8 * RP);   // partials of a token fit in its D / 2 code bytes
     if (S > smax) S = smax;
     if (S > KB) S = KB;
@@ -762,7 +806,7 @@ respin_status_t respin_boundary_forward(respin_plan_t plan, const void* x, const
       const int grid = tiles < plan->sms ? static_cast<int>(tiles) : plan->sms;
       const uint8_t* yp = ypart;
       void* args[] = {&tmRc, &tmXc, &plan->tm_v, &Nv, &Dv, &S, &yp, &ypitch, &h_out, &scale};
-      e = cudaLaunchKernel(plan->tc_re_fn, dim3(static_cast<unsigned>(grid)), dim3(192), args, plan->tc_re_smem, s);
+      e = cudaLaunchKernel(plan->tc_re_fn, dim3(static_cast<unsigned>(grid)), dim3(320), args, plan->tc_re_smem, s);
       if (e != cudaSuccess) return cuda_fail(e, "boundary_tc_reproject_kernel launch");
     }
     {
