@@ -154,6 +154,13 @@ respin_status_t respin_plan_destroy(respin_plan_t plan);
  *   scale     : fp32 [N] per-token scales (device, 4-byte aligned).
  *   stream    : cudaStream_t.
  * No input may overlap an output. Errors: INVALID_ARG, ALIGNMENT, CUDA.
+ *
+ * Large calls of plans with padded rank 64 / 128 (from 256 tokens) and of
+ * rank-16 / 32 plans at D = 8192 (from 4096 tokens) with an h_out buffer run
+ * as three kernels on the stream (projection, re-projection, codes); until
+ * the last one, q_packed holds partial projections and scale the per-token
+ * amax, so, like every output, they are final only once the call's work on
+ * the stream is complete. Nothing is allocated.
  */
 respin_status_t respin_boundary_forward(respin_plan_t plan, const void* x,
                                         const void* residual, int N,
