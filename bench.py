@@ -69,7 +69,10 @@ def parse_args():
                    help="profiling aid: warm up, then launch one kernel once "
                         "(for ncu captures); prints no bench line")
     p.add_argument("--tokens", type=int, default=None,
-                   help="tokens for --profile-launch (default 2048)")
+                   help="tokens for --profile-launch (default: the workload's)")
+    p.add_argument("--rank", type=int, default=None,
+                   help="rank for --profile-launch (default: the workload's; "
+                        "with --workload llama2_70b the factor plan of that rank)")
     p.add_argument("--workload", default="llama2_7b",
                    choices=["llama2_7b", "llama2_7b_w3a3", "tiny", "decode", "llama2_70b",
                             "llama3_8b_stack"],
@@ -1106,16 +1109,20 @@ def run_profile_launch(args):
     import rotation_post_quantization_b200 as rq
     import workloads as W
 
-    w = W.WORKLOADS[WORKLOAD]
+    name = "llama2_70b" if args.workload == "llama2_70b" else WORKLOAD
+    w = W.WORKLOADS[name]
     N = args.tokens or w.N
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
-    fx = W.workload_fixture(WORKLOAD, N=16)
-    if args.boundary_form == "subspace":
-        Qs, Rs = subspace_of(fx)
-        plan = rq.SubspacePlan(w.D, w.r, Qs.astype(np.float32), Rs.astype(np.float32))
+    if name == "llama2_70b":
+        plan = _plan_for(rq, W, w.D, args.rank or w.r, w.k, w.nu)
     else:
-        plan = rq.Plan(w.D, w.r, fx.U.astype(np.float32), fx.V.astype(np.float32))
+        fx = W.workload_fixture(WORKLOAD, N=16)
+        if args.boundary_form == "subspace":
+            Qs, Rs = subspace_of(fx)
+            plan = rq.SubspacePlan(w.D, w.r, Qs.astype(np.float32), Rs.astype(np.float32))
+        else:
+            plan = rq.Plan(w.D, w.r, fx.U.astype(np.float32), fx.V.astype(np.float32))
     kw = dict(n_outlier=w.n_outlier, outlier_scale=w.outlier_scale, dist=w.dist)
     x = W.activations_bf16_fast(N, w.D, tensor_id=W.TID_X, device="cuda", **kw)
     res = W.activations_bf16_fast(N, w.D, tensor_id=W.TID_RESIDUAL, device="cuda", **kw)

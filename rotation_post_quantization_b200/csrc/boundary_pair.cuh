@@ -5,11 +5,13 @@
 //   y = residual Q ; z = y M^T ; h = (residual + x) + z Q^T   (fp32)
 //   h' = bf16(h) ; amax = max|h'| ; inv = qmax/amax ; q = rint(h' inv)
 //
-// Design (B200; CTA pairs = clusters of 2, 8 warps, two CTAs per SM):
-//  * The two CTAs of a pair split the D columns: CTA c owns the DC = D/2
+// Design (B200; clusters of CS = 2 CTAs (pairs) or 4, 8 warps, two CTAs per
+// SM):
+//  * The CTAs of a cluster split the D columns: CTA c owns the DC = D/CS
 //    columns [c DC, (c+1) DC) of every token; warp w owns DC/8 of them
 //    (NB blocks of 64) in every phase, so each shared-memory block is private
-//    to one warp, which refills it as soon as it is done with it.
+//    to one warp, which refills it as soon as it is done with it. Pairs serve
+//    most calls; clusters of 4 halve each CTA's chain for short calls.
 //  * A round is one tile of T <= 16 tokens (one m16 tile; the host picks T so
 //    that every pair gets the same number of rounds). Each CTA keeps about
 //    110 KB of shared memory and at most 128 registers per thread, so two
@@ -33,10 +35,10 @@
 //    16-byte chunk of a row and the chunks of a quarter-warp fall in distinct
 //    bank groups). z is split into bf16 hi + lo parts.
 //  * The two whole-row dependencies (y needs every column, amax needs every
-//    column) are exchanged by pushing this CTA's partials into the peer's
-//    shared memory with st.async (completion counted on the peer's mbarrier,
-//    polled with a non-blocking test). Partial sums are combined in rank
-//    order, so both CTAs use the identical y and z.
+//    column) are exchanged by pushing this CTA's partials into every other
+//    CTA's shared memory with st.async (completion counted on the receiver's
+//    mbarrier, polled with a non-blocking test). Partial sums are combined in
+//    rank order, so every CTA of the cluster uses the identical y and z.
 //  * Every wait is bounded; after a wait gave up the CTA stores nothing more
 //    and requests no further tensor copies (those in flight are waited for).
 #pragma once
@@ -64,9 +66,10 @@ __host__ __device__ constexpr int pr_channel(int t, int n) {
   return 16 * (n >> 1) + 8 * (t >> 2) + 2 * (t & 3) + (n & 1);
 }
 
-template <int DC>
+template <int DC, int CS = 2>
 struct PrCfg {
   static_assert(DC == 1024 || DC == 2048, "columns per CTA");
+  static_assert(CS == 2 || CS == 4, "CTAs per cluster");
   static constexpr int NB = DC / 512;                          // 64-column blocks per warp
   static constexpr uint32_t kTileBytes = kPrT * DC * 2;        // one 16-row tile
   static constexpr uint32_t kXBytes = 8 * kPrXSlots * kPrBlockBytes;   // x slots of all warps
@@ -74,13 +77,14 @@ struct PrCfg {
   static constexpr int BP = 33;                                // y / M row pitch (floats)
   static constexpr uint32_t oRes = 0;                          // residual tile (h' in place)
   static constexpr uint32_t oX = kTileBytes;                   // x slots [2][8 warps]; partial y [8][16][32] in slot 1
-  static constexpr uint32_t oYpeer = oX + kXBytes;             // [2][16][32] peer's partial y
-  static constexpr uint32_t oY = oYpeer + 2 * kPrT * kPrR * 4; // [16][BP] full y
+  // partials from the other CS - 1 CTAs: slot (src - rank - 1) mod CS
+  static constexpr uint32_t oYpeer = oX + kXBytes;             // [2][CS-1][16][32] partial y
+  static constexpr uint32_t oY = oYpeer + 2 * (CS - 1) * kPrT * kPrR * 4;   // [16][BP] full y
   static constexpr uint32_t oZ = oY + kPrT * BP * 4;           // [16][YP] z
   static constexpr uint32_t oM = oZ + kPrT * YP * 4;           // [32][BP] M
   static constexpr uint32_t oWamax = oM + kPrR * BP * 4;       // [8][16]
-  static constexpr uint32_t oApeer = oWamax + 8 * kPrT * 4;    // [2][16] peer's row maxima
-  static constexpr uint32_t oRinv = oApeer + 2 * kPrT * 4;     // [16]
+  static constexpr uint32_t oApeer = oWamax + 8 * kPrT * 4;    // [2][CS-1][16] row maxima
+  static constexpr uint32_t oRinv = oApeer + 2 * (CS - 1) * kPrT * 4;   // [16]
   static constexpr uint32_t oBars = oRinv + kPrT * 4;  // rbar[8], xbar[8][2], ybar[2], abar[2]
   static constexpr uint32_t kSmem = oBars + 28 * 8 + 1024;     // + alignment slack
   static_assert(8 * kPrT * kPrR * 4 <= kXBytes / 2, "the partial y fits in the slot-1 blocks");
@@ -106,13 +110,13 @@ __device__ __forceinline__ void st_async_f32(uint32_t raddr, float a, uint32_t r
 // swizzle. Pf / Rf: the plan's projection / re-projection fragments of both
 // column halves (pr_pack_frags), 8 uint4 per lane per 64-column block.
 // Mg: M = R_sub - I, fp32 [32][32] row-major (zero padded).
-template <int DC, bool F32OUT>
+template <int DC, bool F32OUT, int CS = 2>
 __global__ void __launch_bounds__(kPrThreads, 2)
 boundary_pair_kernel(const __grid_constant__ CUtensorMap tmR, const __grid_constant__ CUtensorMap tmX,
                      const uint4* __restrict__ Pf, const uint4* __restrict__ Rf, const float* __restrict__ Mg,
                      int N, int D, int T, void* __restrict__ h_out, uint8_t* __restrict__ q_out,
                      float* __restrict__ scale_out, float qmax) {
-  using C = PrCfg<DC>;
+  using C = PrCfg<DC, CS>;
   constexpr int NB = C::NB, YP = C::YP, BP = C::BP;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -120,7 +124,7 @@ boundary_pair_kernel(const __grid_constant__ CUtensorMap tmR, const __grid_const
   uint8_t* smem = smem_raw + (base - raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, q4 = lane & 3;
-  const uint32_t rank = cluster_ctarank(), peer = rank ^ 1u;
+  const uint32_t rank = cluster_ctarank();
   const int cid = static_cast<int>(cluster_id_x()), ncl = static_cast<int>(ncluster_x());
   const int ntiles = (N + T - 1) / T;
   const int rounds = cid < ntiles ? (ntiles - cid + ncl - 1) / ncl : 0;
@@ -199,8 +203,8 @@ boundary_pair_kernel(const __grid_constant__ CUtensorMap tmR, const __grid_const
     const int par = r & 1;
     const uint32_t upar = static_cast<uint32_t>(r >> 1) & 1u;
     if (tid == 0) {
-      mbar_arrive_expect_tx(ybar(par), kPrT * kPrR * 4);
-      mbar_arrive_expect_tx(abar(par), kPrT * 4);
+      mbar_arrive_expect_tx(ybar(par), (CS - 1) * kPrT * kPrR * 4);
+      mbar_arrive_expect_tx(abar(par), (CS - 1) * kPrT * 4);
     }
 
     // ---- projection: this warp's partial y over its NB blocks
@@ -253,8 +257,8 @@ boundary_pair_kernel(const __grid_constant__ CUtensorMap tmR, const __grid_const
     ok = __syncthreads_and(ok) != 0;
     if (ok && r + 1 < rounds) prefetch(&tmR, r + 1);
 
-    // ---- y over the pair: thread t owns token t/16, r = 2 (t%16), +1; its
-    // partial (warps summed in order) goes to the peer
+    // ---- y over the cluster: thread t owns token t/16, r = 2 (t%16), +1;
+    // its partial (warps summed in order) goes to every other CTA
     const int yt = tid >> 4, yc = 2 * (tid & 15);
     {
       float2 ys = make_float2(0.f, 0.f);
@@ -268,11 +272,23 @@ boundary_pair_kernel(const __grid_constant__ CUtensorMap tmR, const __grid_const
       // the ring is refilled by tensor copies once every thread is past here
       fence_proxy_async_smem();
       if (!cluster_waited) { cluster_wait(); cluster_waited = true; }
-      st_async_f32x2(map_to_rank(base + C::oYpeer + ((par * kPrT + yt) * kPrR + yc) * 4, peer), ys.x, ys.y,
-                     map_to_rank(ybar(par), peer));
+#pragma unroll
+      for (int p = 1; p < CS; ++p) {   // to CTA rank + p, into its slot CS - 1 - p
+        const uint32_t dst = (rank + p) % CS;
+        const uint32_t yslot = base + C::oYpeer + (((par * (CS - 1) + (CS - 1 - p)) * kPrT + yt) * kPrR + yc) * 4;
+        st_async_f32x2(map_to_rank(yslot, dst), ys.x, ys.y, map_to_rank(ybar(par), dst));
+      }
       ok = mbar_spin_cluster(ybar(par), upar, kSitePairPeer) && ok;
-      const float2 v = *reinterpret_cast<const float2*>(ypeer + (par * kPrT + yt) * kPrR + yc);
-      const float2 y = rank == 0 ? make_float2(ys.x + v.x, ys.y + v.y) : make_float2(v.x + ys.x, v.y + ys.y);
+      // y = sum of the CS partials in rank order
+      float2 y = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int src = 0; src < CS; ++src) {
+        const int sl = (src - static_cast<int>(rank) - 1 + CS) % CS;   // sender's slot here
+        const float2 v = src == static_cast<int>(rank)
+                             ? ys
+                             : *reinterpret_cast<const float2*>(ypeer + ((par * (CS - 1) + sl) * kPrT + yt) * kPrR + yc);
+        if (src == 0) y = v; else { y.x += v.x; y.y += v.y; }
+      }
       ybuf[yt * BP + yc] = y.x;
       ybuf[yt * BP + yc + 1] = y.y;
     }
@@ -378,7 +394,7 @@ boundary_pair_kernel(const __grid_constant__ CUtensorMap tmR, const __grid_const
       else if (ok && s == 0 && r + 1 < rounds) issue_x(r + 1, 0);
     }
 
-    // ---- row amax over the warps, then over the pair
+    // ---- row amax over the warps, then over the cluster
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
       float m = fmaxf(bf16_lo_f32(amax2[hh]), bf16_hi_f32(amax2[hh]));
@@ -391,9 +407,15 @@ boundary_pair_kernel(const __grid_constant__ CUtensorMap tmR, const __grid_const
       float m = 0.f;
 #pragma unroll
       for (int w = 0; w < 8; ++w) m = fmaxf(m, wamax[w * kPrT + tid]);
-      st_async_f32(map_to_rank(base + C::oApeer + (par * kPrT + tid) * 4, peer), m, map_to_rank(abar(par), peer));
+#pragma unroll
+      for (int p = 1; p < CS; ++p) {
+        const uint32_t dst = (rank + p) % CS;
+        const uint32_t aslot = base + C::oApeer + ((par * (CS - 1) + (CS - 1 - p)) * kPrT + tid) * 4;
+        st_async_f32(map_to_rank(aslot, dst), m, map_to_rank(abar(par), dst));
+      }
       ok = mbar_spin_cluster(abar(par), upar, kSitePairPeer) && ok;
-      m = fmaxf(m, apeer[par * kPrT + tid]);
+#pragma unroll
+      for (int sl = 0; sl < CS - 1; ++sl) m = fmaxf(m, apeer[(par * (CS - 1) + sl) * kPrT + tid]);
       float inv, sc;
       inv_and_scale(m, qmax, inv, sc);
       rowinv[tid] = inv;
@@ -421,7 +443,7 @@ boundary_pair_kernel(const __grid_constant__ CUtensorMap tmR, const __grid_const
     if (ok && r + 1 < rounds) issue_res(r + 1);
   }
   if (!cluster_waited) cluster_wait();   // no round: close the set-up barrier phase
-  // neither CTA may leave while the peer can still push into it
+  // no CTA may leave while another can still push into it
   cluster_sync();
 }
 

@@ -104,6 +104,10 @@ struct respin_plan_s {
   const void* pair_fn = nullptr;
   size_t pair_smem = 0;
   int pair_max = 0;              // co-resident CTA pairs
+  // Clusters of 4 (D = 4096: a quarter of the columns per CTA) for short calls.
+  const void* quad_fn = nullptr;
+  size_t quad_smem = 0;
+  int quad_max = 0;              // co-resident 4-CTA clusters
   // Tensor-core passes for padded ranks 64 / 128 (boundary_tc.cuh): tensor
   // maps of the plan's U^T [r_pad, D] and V [D, r_pad] (the factor layout of
   // the shared-memory cluster kernel).
@@ -439,9 +443,9 @@ respin_status_t configure_boundary(int D, int R, bool f32, BoundaryConfig* out, 
               "no cluster configuration holds the factor slices for D=%d, padded r=%d", D, R);
 }
 
-template <int DC, bool F32>
+template <int DC, bool F32, int CS = 2>
 const void* pair_fn() {
-  return reinterpret_cast<const void*>(&boundary_pair_kernel<DC, F32>);
+  return reinterpret_cast<const void*>(&boundary_pair_kernel<DC, F32, CS>);
 }
 
 // The pair kernel for D columns (D / 2 per CTA) and its co-resident pairs.
@@ -458,6 +462,17 @@ respin_status_t configure_pair(int D, bool f32, respin_plan_s* p) {
   p->pair_fn = fn;
   p->pair_smem = smem;
   p->pair_max = n;
+  if (D == 4096) {   // clusters of 4 for short calls (optional)
+    const void* qf = f32 ? pair_fn<1024, true, 4>() : pair_fn<1024, false, 4>();
+    const size_t qs = PrCfg<1024, 4>::kSmem;
+    const int nq = max_active_clusters(qf, 4, qs, kPrThreads);
+    if (nq > 0) {
+      p->quad_fn = qf;
+      p->quad_smem = qs;
+      p->quad_max = nq;
+    }
+    cudaGetLastError();
+  }
   return ok();
 }
 
@@ -739,6 +754,32 @@ respin_status_t respin_boundary_forward(respin_plan_t plan, const void* x, const
     // chosen so that every pair gets the same number of tiles (two CTAs per
     // SM share the work evenly).
     const long long tiles16 = (static_cast<long long>(N) + kPrT - 1) / kPrT;
+    if (plan->quad_fn != nullptr && tiles16 <= plan->quad_max / 2) {
+      // short call: clusters of 4, full 16-token tiles, at most one CTA per SM
+      CUtensorMap tmR, tmX;
+      if (!make_tmap_bf16_tile(&tmR, residual, N, D, kPrT) || !make_tmap_bf16_tile(&tmX, x, N, D, kPrT))
+        return fail(RESPIN_ERR_CUDA, "cuTensorMapEncodeTiled failed for the residual / x tiles");
+      const uint4* pf = reinterpret_cast<const uint4*>(plan->q_pair);
+      const uint4* rf = reinterpret_cast<const uint4*>(plan->q_pair + static_cast<size_t>(D) * kPrR / 2);
+      const float* mg = plan->m_pair;
+      int Dv = D, Tq = kPrT;
+      void* args[] = {&tmR, &tmX, &pf, &rf, &mg, &N, &Dv, &Tq, &h_out, &q_packed, &scale, &qmax};
+      cudaLaunchConfig_t lc = {};
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 4;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      lc.gridDim = dim3(static_cast<unsigned>(4 * tiles16), 1, 1);
+      lc.blockDim = dim3(kPrThreads, 1, 1);
+      lc.dynamicSmemBytes = plan->quad_smem;
+      lc.stream = s;
+      lc.attrs = attr;
+      lc.numAttrs = 1;
+      cudaError_t e = cudaLaunchKernelExC(&lc, plan->quad_fn, args);
+      if (e != cudaSuccess) return cuda_fail(e, "boundary_pair_kernel (clusters of 4) launch");
+      return ok();
+    }
     int T = kPrT;
     if (tiles16 > plan->pair_max / 2) {
       const long long per = static_cast<long long>(plan->pair_max) * kPrT;
