@@ -18,8 +18,9 @@
 //     B = the tile's rows of V: two tcgen05 MMA chains into one TMEM
 //     accumulator give y V^T. The epilogue adds residual + x (32-column
 //     chunks by tensor copies, 64-byte swizzle), rounds to bf16, writes h'
-//     and folds the tile's row maxima of |h'| into the scale buffer with an
-//     atomic max (non-negative floats order like their bit patterns).
+//     over the chunk's residual rows and out by tensor stores, and folds the
+//     tile's row maxima of |h'| into the scale buffer with an atomic max
+//     (non-negative floats order like their bit patterns).
 //  3. boundary_quant_rows_kernel: codes and scales of every token from h' and
 //     its amax.
 //
@@ -189,6 +190,7 @@ struct TcReCfg {
 };
 
 // tmRc / tmXc: residual / x bf16 [N, D], box {32, 128}, 64-byte swizzle.
+// tmH: h_out bf16 [N, D], box {32, 32}, 64-byte swizzle (unused for fp32 h).
 // tmV: V bf16 [D, RP], box {64, 128}, 128-byte swizzle. Tiles t = m * (D /
 // 128) + n (token tile m, column tile n); CTA b takes the contiguous range
 // [b T / G, (b+1) T / G). amax: the scale buffer, zero on entry, receives
@@ -196,7 +198,8 @@ struct TcReCfg {
 template <int RP, bool F32OUT>
 __global__ void __launch_bounds__(320, 1)
 boundary_tc_reproject_kernel(const __grid_constant__ CUtensorMap tmRc, const __grid_constant__ CUtensorMap tmXc,
-                             const __grid_constant__ CUtensorMap tmV, int N, int D, int S,
+                             const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUtensorMap tmV,
+                             int N, int D, int S,
                              const uint8_t* __restrict__ ypart, int ypitch, void* __restrict__ h_out,
                              float* __restrict__ amax) {
   using C = TcReCfg<RP>;
@@ -367,17 +370,25 @@ boundary_tc_reproject_kernel(const __grid_constant__ CUtensorMap tmRc, const __g
       if (ok) ok = mbar_wait(afull(ab), (i >> 1) & 1, kSiteTcAccum);
       ok = __all_sync(0xffffffffu, ok);
       tc_fence_after();
+      // both chunks' accumulators at once, then the buffer goes back to the
+      // MMA issuer
+      uint32_t v[2][32];
+      const uint32_t tb = tmem + (static_cast<uint32_t>(32 * qd) << 16) + ab * kTcBN + kTcChunk * 2 * half;
+      tmem_ld_32x32b_x32(tb, v[0]);
+      tmem_ld_32x32b_x32(tb + kTcChunk, v[1]);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(aempty(ab));
       float rmax = 0.f;
-#pragma unroll 1
-      for (int c = 2 * half; c < 2 * half + 2; ++c) {
-        const int pidx = 2 * i + (c - 2 * half);   // position in this half's chunk ring
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+        const int c = 2 * half + cc;
+        const int pidx = 2 * i + cc;   // position in this half's chunk ring
         const int cs = half * C::HST + pidx % C::HST;
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(32 * qd) << 16) + ab * kTcBN + kTcChunk * c, v);
-        tmem_wait_ld();
         if (ok) ok = mbar_wait(cfull(cs), (pidx / C::HST) & 1, kSiteTcLoad);
         ok = __all_sync(0xffffffffu, ok);
-        const uint8_t* rs = smem + C::oC + cs * C::CBytes;
+        uint8_t* rs = smem + C::oC + cs * C::CBytes;
         const uint8_t* xs = rs + C::CHalf;
         uint4 rv[4], xv[4];
 #pragma unroll
@@ -385,12 +396,7 @@ boundary_tc_reproject_kernel(const __grid_constant__ CUtensorMap tmRc, const __g
           rv[j] = *reinterpret_cast<const uint4*>(rs + tc_sw64(r, j));
           xv[j] = *reinterpret_cast<const uint4*>(xs + tc_sw64(r, j));
         }
-        // the stage's bytes are read (generic proxy) before its next copy
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(cempty(cs));
         const size_t gcol = static_cast<size_t>(n) * kTcBN + kTcChunk * c;
-        const bool store = ok && tok < N;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const uint32_t rw[4] = {rv[j].x, rv[j].y, rv[j].z, rv[j].w}, xw[4] = {xv[j].x, xv[j].y, xv[j].z, xv[j].w};
@@ -399,29 +405,46 @@ boundary_tc_reproject_kernel(const __grid_constant__ CUtensorMap tmRc, const __g
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const float2 sum = add_f32x2(bf16x2_to_f32x2(rw[e]), bf16x2_to_f32x2(xw[e]));
-            const float2 acc = make_float2(__uint_as_float(v[8 * j + 2 * e]), __uint_as_float(v[8 * j + 2 * e + 1]));
+            const float2 acc =
+                make_float2(__uint_as_float(v[cc][8 * j + 2 * e]), __uint_as_float(v[cc][8 * j + 2 * e + 1]));
             hf[e] = add_f32x2(sum, acc);
             hw[e] = pack_bf16x2(hf[e].x, hf[e].y);
             rmax = fmaxf(rmax, fmaxf(fabsf(bf16_lo_f32(hw[e])), fabsf(bf16_hi_f32(hw[e]))));
           }
-          if (store) {
-            if constexpr (F32OUT) {
-              float4* hp = reinterpret_cast<float4*>(static_cast<float*>(h_out) + static_cast<size_t>(tok) * D + gcol + 8 * j);
+          if constexpr (F32OUT) {
+            if (ok && tok < N) {
+              float4* hp =
+                  reinterpret_cast<float4*>(static_cast<float*>(h_out) + static_cast<size_t>(tok) * D + gcol + 8 * j);
               hp[0] = make_float4(hf[0].x, hf[0].y, hf[1].x, hf[1].y);
               hp[1] = make_float4(hf[2].x, hf[2].y, hf[3].x, hf[3].y);
-            } else {
-              *reinterpret_cast<uint4*>(static_cast<bf16*>(h_out) + static_cast<size_t>(tok) * D + gcol + 8 * j) =
-                  make_uint4(hw[0], hw[1], hw[2], hw[3]);
             }
+          } else {
+            // h' over this thread's own residual row of the stage
+            *reinterpret_cast<uint4*>(rs + tc_sw64(r, j)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
           }
         }
+        // generic-proxy accesses of the stage before the tensor store reads
+        // it and before its next copy
+        fence_proxy_async_smem();
+        __syncwarp();
+        if constexpr (!F32OUT) {
+          // this warp's 32 rows of h' go out as one tensor store (rows past N
+          // are clipped); the stage is released once the store has read them
+          const int y0 = tile_m(i) * kTcBM + 32 * qd;
+          if (lane == 0 && ok && y0 < N) {
+            tma_store_2d(&tmH, static_cast<int>(gcol), y0, base + C::oC + cs * C::CBytes + 32 * qd * 64);
+            bulk_commit_group();
+            bulk_wait_group_read<0>();
+          }
+          __syncwarp();
+        }
+        if (lane == 0) mbar_arrive(cempty(cs));
       }
-      // the accumulator buffer goes back to the MMA issuer
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(aempty(ab));
       if (ok && tok < N) atomicMax(reinterpret_cast<unsigned int*>(amax) + tok, __float_as_uint(rmax));
     }
+    // every h' tensor store of this warp has completed before the launch ends
+    if (lane == 0) bulk_wait_group_all();
+    __syncwarp();
     if (!ok) *abort_flag = 1;
   }
   __syncthreads();

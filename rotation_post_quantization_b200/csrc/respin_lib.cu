@@ -827,11 +827,13 @@ respin_status_t respin_boundary_forward(respin_plan_t plan, const void* x, const
     if (S > KB) S = KB;
     if (S > 8) S = 8;
     if (S < 1) S = 1;
-    CUtensorMap tmR, tmRc, tmXc;
+    CUtensorMap tmR, tmRc, tmXc, tmH;
     if (!make_tmap_bf16(&tmR, residual, N, D, 64, kTcBM, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_tmap_bf16(&tmRc, residual, N, D, kTcChunk, kTcBM, CU_TENSOR_MAP_SWIZZLE_64B) ||
-        !make_tmap_bf16(&tmXc, x, N, D, kTcChunk, kTcBM, CU_TENSOR_MAP_SWIZZLE_64B))
+        !make_tmap_bf16(&tmXc, x, N, D, kTcChunk, kTcBM, CU_TENSOR_MAP_SWIZZLE_64B) ||
+        (!f32 && !make_tmap_bf16(&tmH, h_out, N, D, kTcChunk, 32, CU_TENSOR_MAP_SWIZZLE_64B)))
       return fail(RESPIN_ERR_CUDA, "cuTensorMapEncodeTiled failed for the tensor-core boundary tiles");
+    if (f32) tmH = tmRc;   // not used by the fp32-h variant
     cudaError_t e = cudaMemsetAsync(scale, 0, static_cast<size_t>(N) * sizeof(float), s);
     if (e != cudaSuccess) return cuda_fail(e, "clearing the scale buffer");
     uint8_t* ypart = static_cast<uint8_t*>(q_packed);
@@ -846,7 +848,7 @@ respin_status_t respin_boundary_forward(respin_plan_t plan, const void* x, const
       const long long tiles = static_cast<long long>(mtiles) * (D / kTcBN);
       const int grid = tiles < plan->sms ? static_cast<int>(tiles) : plan->sms;
       const uint8_t* yp = ypart;
-      void* args[] = {&tmRc, &tmXc, &plan->tm_v, &Nv, &Dv, &S, &yp, &ypitch, &h_out, &scale};
+      void* args[] = {&tmRc, &tmXc, &tmH, &plan->tm_v, &Nv, &Dv, &S, &yp, &ypitch, &h_out, &scale};
       e = cudaLaunchKernel(plan->tc_re_fn, dim3(static_cast<unsigned>(grid)), dim3(320), args, plan->tc_re_smem, s);
       if (e != cudaSuccess) return cuda_fail(e, "boundary_tc_reproject_kernel launch");
     }
