@@ -23,6 +23,10 @@
 //     (non-negative floats order like their bit patterns).
 //  3. boundary_quant_rows_kernel: codes and scales of every token from h' and
 //     its amax.
+// Passes 2 and 3 are launched as programmatic dependents: a pass starts while
+// the previous one finishes (pass 2 streams residual, x and V at once) and
+// waits for the previous pass's results only where it reads them. Pass 1
+// clears the amax accumulators.
 //
 // HBM traffic per token: residual twice, x once, h' written and read back,
 // codes and scale: 10 D + 4 bytes (8.5 D + 4 for h' in fp32 aside), against
@@ -74,7 +78,8 @@ struct TcProjCfg {
 template <int RP>
 __global__ void __launch_bounds__(128, 1)
 boundary_tc_project_kernel(const __grid_constant__ CUtensorMap tmR, const __grid_constant__ CUtensorMap tmU,
-                           int N, int KB, int S, uint8_t* __restrict__ ypart, int ypitch) {
+                           int N, int KB, int S, uint8_t* __restrict__ ypart, int ypitch,
+                           float* __restrict__ amax) {
   using C = TcProjCfg<RP>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -100,6 +105,10 @@ boundary_tc_project_kernel(const __grid_constant__ CUtensorMap tmR, const __grid
     asm volatile("prefetch.tensormap [%0];" ::"l"(&tmU) : "memory");
   }
   if (warp == 0) { tmem_alloc(tslot, RP); tmem_relinquish(); }
+  // the re-projection pass may start its independent work now
+  grid_dep_launch();
+  // the amax accumulator of this token tile starts at zero (bit pattern 0)
+  if (split == 0 && m0 + tid < N) amax[m0 + tid] = 0.0f;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -242,6 +251,7 @@ boundary_tc_reproject_kernel(const __grid_constant__ CUtensorMap tmRc, const __g
     asm volatile("prefetch.tensormap [%0];" ::"l"(&tmV) : "memory");
   }
   if (warp == 0) { tmem_alloc(tslot, 2 * kTcBN); tmem_relinquish(); }
+  grid_dep_launch();   // the code pass may be scheduled (it waits for this grid)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -326,6 +336,10 @@ boundary_tc_reproject_kernel(const __grid_constant__ CUtensorMap tmRc, const __g
     const int qd = warp & 3;
     const int half = (warp - 2) >> 2;
     const int r = 32 * qd + lane;
+    // the partial y and the zeroed amax come from the projection pass, which
+    // may still be running (the tensor copies of residual, x and V need not
+    // wait for it)
+    grid_dep_wait();
     int seg = 0;
     bool ok = true;
     for (int i = 0; i < nloc && ok; ++i) {
@@ -470,6 +484,7 @@ boundary_quant_rows_kernel(const void* __restrict__ h, int N, int D, uint8_t* __
   constexpr int VPT = 8;   // 16-byte vectors of h' per thread per pass (D <= 16384 in one pass)
   const int tid = threadIdx.x;
   const int nv = D / 8;
+  grid_dep_wait();   // h' and amax come from the re-projection pass
   for (int row = blockIdx.x; row < N; row += gridDim.x) {
     const float amax = scale_io[row];
     float inv, sc;

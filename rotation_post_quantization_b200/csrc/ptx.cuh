@@ -172,6 +172,21 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
                : "memory");
 }
 
+// ---------------------------------------------------------------- dependent launches
+
+// Programmatic dependent launch: a kernel launched with the programmatic
+// stream-serialization attribute may start while the previous kernel of the
+// stream still runs; grid_dep_wait() blocks until that kernel has completed
+// and its memory operations are visible. grid_dep_launch() lets the next
+// such kernel start before this one ends. Both are no-ops for kernels
+// launched without the attribute.
+__device__ __forceinline__ void grid_dep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dep_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- async proxy
 
 __device__ __forceinline__ void fence_proxy_async_smem() {

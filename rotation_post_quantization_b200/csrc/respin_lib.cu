@@ -215,6 +215,23 @@ const void* tc_re_fn() {
   return reinterpret_cast<const void*>(&boundary_tc_reproject_kernel<RP, F32>);
 }
 
+// A launch that may begin while the previous kernel of the stream finishes
+// (programmatic stream serialization); the kernel waits for that kernel's
+// results itself (grid_dep_wait).
+cudaError_t launch_dependent(const void* fn, int grid, int block, size_t smem, cudaStream_t s, void** args) {
+  cudaLaunchConfig_t lc = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  lc.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+  lc.blockDim = dim3(static_cast<unsigned>(block), 1, 1);
+  lc.dynamicSmemBytes = smem;
+  lc.stream = s;
+  lc.attrs = attr;
+  lc.numAttrs = 1;
+  return cudaLaunchKernelExC(&lc, fn, args);
+}
+
 // The tensor-core passes of a plan: padded rank 64 / 128 (factors already
 // stored as U^T then V), or padded rank 16 / 32 on the register-factor
 // cluster kernel (D = 8192 and other widths the row-tile kernel does not
@@ -834,12 +851,11 @@ respin_status_t respin_boundary_forward(respin_plan_t plan, const void* x, const
         (!f32 && !make_tmap_bf16(&tmH, h_out, N, D, kTcChunk, 32, CU_TENSOR_MAP_SWIZZLE_64B)))
       return fail(RESPIN_ERR_CUDA, "cuTensorMapEncodeTiled failed for the tensor-core boundary tiles");
     if (f32) tmH = tmRc;   // not used by the fp32-h variant
-    cudaError_t e = cudaMemsetAsync(scale, 0, static_cast<size_t>(N) * sizeof(float), s);
-    if (e != cudaSuccess) return cuda_fail(e, "clearing the scale buffer");
+    cudaError_t e;
     uint8_t* ypart = static_cast<uint8_t*>(q_packed);
     int ypitch = D / 2, Nv = N, Dv = D;
     {
-      void* args[] = {&tmR, &plan->tm_ut, &Nv, &KB, &S, &ypart, &ypitch};
+      void* args[] = {&tmR, &plan->tm_ut, &Nv, &KB, &S, &ypart, &ypitch, &scale};
       e = cudaLaunchKernel(plan->tc_proj_fn, dim3(static_cast<unsigned>(mtiles * S)), dim3(128), args,
                            plan->tc_proj_smem, s);
       if (e != cudaSuccess) return cuda_fail(e, "boundary_tc_project_kernel launch");
@@ -849,14 +865,18 @@ respin_status_t respin_boundary_forward(respin_plan_t plan, const void* x, const
       const int grid = tiles < plan->sms ? static_cast<int>(tiles) : plan->sms;
       const uint8_t* yp = ypart;
       void* args[] = {&tmRc, &tmXc, &tmH, &plan->tm_v, &Nv, &Dv, &S, &yp, &ypitch, &h_out, &scale};
-      e = cudaLaunchKernel(plan->tc_re_fn, dim3(static_cast<unsigned>(grid)), dim3(320), args, plan->tc_re_smem, s);
+      e = launch_dependent(plan->tc_re_fn, grid, 320, plan->tc_re_smem, s, args);
       if (e != cudaSuccess) return cuda_fail(e, "boundary_tc_reproject_kernel launch");
     }
     {
       const int grid = N < plan->sms * 8 ? N : plan->sms * 8;
-      if (f32) boundary_quant_rows_kernel<true><<<grid, 256, 0, s>>>(h_out, N, D, q_packed, scale, qmax);
-      else boundary_quant_rows_kernel<false><<<grid, 256, 0, s>>>(h_out, N, D, q_packed, scale, qmax);
-      e = cudaGetLastError();
+      const void* hq = h_out;
+      uint8_t* qp = q_packed;
+      float* sp = scale;
+      void* args[] = {&hq, &Nv, &Dv, &qp, &sp, &qmax};
+      e = launch_dependent(f32 ? reinterpret_cast<const void*>(&boundary_quant_rows_kernel<true>)
+                               : reinterpret_cast<const void*>(&boundary_quant_rows_kernel<false>),
+                           grid, 256, 0, s, args);
       if (e != cudaSuccess) return cuda_fail(e, "boundary_quant_rows_kernel launch");
     }
     return ok();
