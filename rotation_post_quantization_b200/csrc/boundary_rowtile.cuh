@@ -172,6 +172,11 @@ boundary_rowtile_kernel(const __grid_constant__ CUtensorMap tmR, const __grid_co
     }
   }
   __syncwarp();
+  // launched as a programmatic dependent: residual and x may come from the
+  // previous kernel of the stream, so every global access waits for it; the
+  // next kernel (the GEMM on these codes) may be scheduled from here on
+  grid_dep_wait();
+  grid_dep_launch();
 
   // x block stream of this warp: use u is block u % NB of the warp's slice in
   // its tile iteration u / NB, staged in slot u % XS by lane u % XS.

@@ -895,7 +895,7 @@ respin_status_t respin_boundary_forward(respin_plan_t plan, const void* x, const
     const uint4* vt = reinterpret_cast<const uint4*>(fac + static_cast<size_t>(plan->r_pad) * D);
     const int grid = ntiles < c.max_clusters ? ntiles : c.max_clusters;
     void* args[] = {&tmR, &tmX, &ut, &vt, &N, &h_out, &q_packed, &scale, &qmax};
-    cudaError_t e = cudaLaunchKernel(c.fn, dim3(grid), dim3(32 * c.cluster), args, c.smem, s);
+    cudaError_t e = launch_dependent(c.fn, grid, 32 * c.cluster, c.smem, s, args);
     if (e != cudaSuccess) return cuda_fail(e, "boundary_rowtile_kernel launch");
     return ok();
   }
@@ -1053,17 +1053,21 @@ static respin_status_t gemm_common(const uint8_t* q_act, const float* scale_act,
   const long long groups = CG == 2 ? (tiles < info.max_pairs ? tiles : info.max_pairs)
                                    : (tiles < info.sms ? tiles : info.sms);
   cudaLaunchConfig_t lc = {};
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = CG;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  // programmatic dependent: set-up overlaps the previous kernel's tail; the
+  // kernel waits for it before its first global access
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   lc.gridDim = dim3(static_cast<unsigned>(groups * CG), 1, 1);
   lc.blockDim = dim3(kGemmThreads, 1, 1);
   lc.dynamicSmemBytes = CG == 2 ? GemmCfg<2>::Smem : GemmCfg<1>::Smem;
   lc.stream = s;
   lc.attrs = attr;
-  lc.numAttrs = 1;
+  lc.numAttrs = 2;
   void* args[] = {&tmA, &tmB, &tmO, const_cast<float**>(&scale_act), const_cast<float**>(&scale_w), &N, &K, &O};
   e = cudaLaunchKernelExC(&lc, fn, args);
   if (e != cudaSuccess) return cuda_fail(e, "w4a4_gemm_kernel launch");

@@ -181,6 +181,7 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   tc_fence_before();
   if constexpr (CG == 2) cluster_sync(); else __syncthreads();
   tc_fence_after();
+  grid_dep_launch();   // the next kernel of the stream may be scheduled
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + (tslot - base));
   // barriers signalled in the leader CTA by both CTAs of the pair
   const uint32_t full_leader0 = CG == 2 ? map_to_rank(full0, 0) : full0;
@@ -305,6 +306,9 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     }
   } else if (warp == kGemmTmaWarp) {
     // ------------------------------------------------ TMA warp: packed K blocks
+    // launched as a programmatic dependent: the codes (and possibly the
+    // weights) come from earlier kernels of the stream
+    grid_dep_wait();
     if (lane < 2 * G::PS) {
       const int stage = lane >> 1;
       const bool is_b = (lane & 1) != 0;
@@ -373,6 +377,7 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     // row segment reaches L2 as whole sectors. int32 output takes two units
     // (16 columns each) per chunk.
     float* sws = reinterpret_cast<float*>(smem + (swbase - base) + quad * G::SwBytes);
+    grid_dep_wait();   // the activation scales and the output buffer
     bool ok = true;
     int local = 0;
     for (int t = group; t < tiles; t += ngroups, ++local) {
