@@ -992,9 +992,13 @@ def wl_stack(args, env, form: str, cpu: bool) -> dict:
     xm = torch.empty(N, D, dtype=torch.bfloat16, device=env.dev)
     _, q3, s3, _ = env.outs(N, D)
     qonly = rq.Plan(M, 0)
+    rowmax = torch.empty(N, M // 256, dtype=torch.float32, device=env.dev)
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(5 * L + 1)]
     sp = env.sptr
 
+    # The up projection's GEMM also writes the per-token maxima of its output
+    # per 256-channel tile, so the quant-only step before the down projection
+    # is a pure streaming pass (no reduction of its own).
     def stack(record):
         cur = res0
         for l in range(L):
@@ -1002,9 +1006,9 @@ def wl_stack(args, env, form: str, cpu: bool) -> dict:
             if record: ev[5 * l].record(env.stream)
             rq.respin_boundary_forward(plans[2 * l], xatt[l % 4], cur, h1, q1, s1, sp)
             if record: ev[5 * l + 1].record(env.stream)
-            rq.w4a4_gemm(q1, s1, wup[l][0], wup[l][1], u, sp)
+            rq.w4a4_gemm_rowmax(q1, s1, wup[l][0], wup[l][1], u, rowmax, sp)
             if record: ev[5 * l + 2].record(env.stream)
-            rq.respin_boundary_forward(qonly, u, None, None, q2, s2, sp)
+            rq.respin_quantize_rowmax(u, rowmax, q2, s2, 0, sp)
             if record: ev[5 * l + 3].record(env.stream)
             rq.w4a4_gemm(q2, s2, wdn[l][0], wdn[l][1], xm, sp)
             if record: ev[5 * l + 4].record(env.stream)
@@ -1017,10 +1021,22 @@ def wl_stack(args, env, form: str, cpu: bool) -> dict:
     reps = 3
     parts = np.zeros(5)
     total = 0.0
-    for _ in range(reps):
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    for _ in range(reps):   # the stack alone (no events between its kernels)
+        t0.record(env.stream)
+        stack(False)
+        t1.record(env.stream)
+        torch.cuda.synchronize()
+        total += t0.elapsed_time(t1)
+    # the quant-only step as a row-wise pass with its own reduction, for comparison
+    for _ in range(3):
+        rq.respin_boundary_forward(qonly, u, None, None, q2, s2, sp)
+    qo_rowwise_us = _events_ms(torch, lambda i: rq.respin_boundary_forward(qonly, u, None, None, q2, s2, sp),
+                               10, env.stream) * 1e3
+    for _ in range(reps):   # per-part device times (events between the kernels)
         stack(True)
         torch.cuda.synchronize()
-        total += ev[0].elapsed_time(ev[5 * L])
         for l in range(L):
             for j in range(5):
                 parts[j] += ev[5 * l + j].elapsed_time(ev[5 * l + j + 1])
@@ -1035,11 +1051,16 @@ def wl_stack(args, env, form: str, cpu: bool) -> dict:
     bb = boundary_bytes(N, D, w.r, form)
     out = {"config": {"D": D, "N": N, "layers": L, "mlp": M, "r": w.r,
                       "plan": "stored subspace form" if form == "subspace" else "factor pair",
-                      "chain": "attn boundary, GEMM D->mlp, quant-only mlp, GEMM mlp->D, mlp boundary "
+                      "chain": "attn boundary, GEMM D->mlp (with per-token tile maxima of its output), "
+                               "quant-only mlp from those maxima, GEMM mlp->D, mlp boundary "
                                "(nonlinearity omitted)"},
            "tokens_per_s": N / (ms * 1e-3), "ms_per_stack": ms,
            "per_layer_us": {"attn_boundary": parts[0], "gemm_up": parts[1], "quant_only": parts[2],
                             "gemm_down": parts[3], "mlp_boundary": parts[4]},
+           "quant_only_rowwise_us": qo_rowwise_us,
+           "note": "ms_per_stack: the stack with no events between its kernels; per_layer_us: "
+                   "the same stack with events around every kernel; quant_only_rowwise_us: the "
+                   "quant-only step as a row-wise pass with its own reduction, for comparison",
            "gemm_tops": ops / ((parts[1] + parts[3]) * L * 1e-6) / 1e12,
            "boundary_frac_of_hbm": bb / env.hbm_gbs / 1e3 / ((parts[0] + parts[4]) / 2),
            "quant_only_frac_of_hbm": (N * (2 * M + M / 2 + 4)) / env.hbm_gbs / 1e3 / parts[2]}

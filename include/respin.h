@@ -23,7 +23,7 @@
  *     device that is current when the call is made, 16-byte aligned unless
  *     stated otherwise. The library never allocates per call.
  *   - `stream` is a cudaStream_t handle (NULL = legacy default stream). Calls
- *     are asynchronous: they validate, enqueue one kernel and return.
+ *     are asynchronous: they validate, enqueue their kernels and return.
  *   - Every call returns a respin_status_t. Validation errors are returned
  *     before anything is enqueued; respin_last_error() then holds a message.
  *     Kernels never trap: a kernel that gives up on a bounded wait records a
@@ -103,8 +103,8 @@ respin_status_t respin_plan_create(respin_plan_t* out, int D, int r,
  * i.e. the factor form with U_r = Q and V_r = Q M, stored in half the bytes.
  *
  *   out    : receives the plan handle.
- *   D      : hidden size; 2048 or 4096 (the two CTAs of a pair each hold
- *            half of Q on chip).
+ *   D      : hidden size; 2048 or 4096 (CTA pairs split the columns;
+ *            short calls at D = 4096 use clusters of four).
  *   r      : rank, 1 <= r <= 32.
  *   Q      : HOST fp32 [D, r] row-major.
  *   R_sub  : HOST fp32 [r, r] row-major.
@@ -195,6 +195,48 @@ respin_status_t w4a4_gemm(const uint8_t* q_act, const float* scale_act,
 respin_status_t w4a4_gemm_i32(const uint8_t* q_act, const uint8_t* q_w,
                               int N, int K, int O, int32_t* acc_out,
                               void* stream);
+
+/*
+ * w4a4_gemm_rowmax -- w4a4_gemm, and in the same pass the maxima of |out|
+ * (out as stored, bf16) per token and 256-channel tile:
+ *     rowmax[n, t] = max_{o in [256 t, 256 t + 256) and o < O} |out[n, o]|
+ * for a following per-token quantization of out (the input of the next
+ * linear, e.g. the up projection's output feeding the down projection in
+ * the quantized linears of zh §3-§4), so that pass needs no reduction of its
+ * own.
+ *
+ *   rowmax : fp32 [N, ceil(O / 256)] (device, 4-byte aligned, caller-owned;
+ *            every entry is written).
+ *   Other arguments as w4a4_gemm. Needs N > 128 (the tensor-memory kernel);
+ *   smaller N gives UNSUPPORTED. Errors: as w4a4_gemm.
+ */
+respin_status_t w4a4_gemm_rowmax(const uint8_t* q_act, const float* scale_act,
+                                 const uint8_t* q_w, const float* scale_w,
+                                 int N, int K, int O, void* out,
+                                 float* rowmax, void* stream);
+
+/*
+ * respin_quantize_rowmax -- per-token codes and scales of a bf16 matrix u
+ * [N, D] whose per-token maxima of |u| are given as partial maxima (rowmax
+ * [N, D / 256], as written by w4a4_gemm_rowmax): amax = max over the row's
+ * partials, then the quantizer of respin_boundary_forward (inv = B / amax,
+ * scale = amax / B, q = rint(u inv), B = 7, or 3 with RESPIN_ACT_INT3;
+ * amax < 2^-125 gives scale 0 and zero codes). The codes equal those of
+ * respin_boundary_forward with an r = 0 plan and no residual on the same u.
+ *
+ *   u        : bf16 [N, D] (device, 16-byte aligned).
+ *   rowmax   : fp32 [N, D / 256] (device).
+ *   N, D     : D % 256 == 0, 256 <= D <= 65536.
+ *   q_packed : uint8 [N, D/2]; scale : fp32 [N] (device).
+ *   flags    : 0 or RESPIN_ACT_INT3.
+ * Launched as a programmatic dependent of the previous kernel of the stream
+ * (it waits for that kernel before reading u). Errors: INVALID_ARG,
+ * UNSUPPORTED, ALIGNMENT, CUDA.
+ */
+respin_status_t respin_quantize_rowmax(const void* u, const float* rowmax,
+                                       int N, int D, uint8_t* q_packed,
+                                       float* scale, unsigned flags,
+                                       void* stream);
 
 /*
  * respin_factors_from_subspace -- plan factors from the subspace form.

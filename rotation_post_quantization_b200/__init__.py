@@ -28,6 +28,7 @@ RESPIN_ACT_INT3 = 2
 # Every entry point include/respin.h declares (checked by the tests).
 EXPORTED = ("respin_plan_create", "respin_plan_create_subspace", "respin_plan_destroy",
             "respin_boundary_forward", "w4a4_gemm", "w4a4_gemm_i32",
+            "w4a4_gemm_rowmax", "respin_quantize_rowmax",
             "respin_factors_from_subspace", "respin_factors_from_transition",
             "respin_fuse_weight", "respin_quantize_weight",
             "respin_device_status", "respin_selftest_wait_limit",
@@ -57,6 +58,8 @@ def _load() -> ctypes.CDLL:
     lib.respin_boundary_forward.argtypes = [vp, vp, vp, i32, vp, vp, vp, vp]
     lib.w4a4_gemm.argtypes = [vp, vp, vp, vp, i32, i32, i32, vp, vp]
     lib.w4a4_gemm_i32.argtypes = [vp, vp, i32, i32, i32, vp, vp]
+    lib.w4a4_gemm_rowmax.argtypes = [vp, vp, vp, vp, i32, i32, i32, vp, vp, vp]
+    lib.respin_quantize_rowmax.argtypes = [vp, vp, i32, i32, vp, vp, u32, vp]
     dp = ctypes.POINTER(ctypes.c_double)
     lib.respin_factors_from_subspace.argtypes = [i32, i32, fp, fp, fp, fp]
     lib.respin_factors_from_transition.argtypes = [i32, i32, fp, ctypes.c_double, fp, fp, dp]
@@ -190,6 +193,24 @@ def w4a4_gemm_i32(q_act, q_w, acc_out, stream=None) -> None:
     O = q_w.shape[0]
     _check(lib.w4a4_gemm_i32(_ptr(q_act), _ptr(q_w), int(N), int(2 * K2),
                              int(O), _ptr(acc_out), _stream(stream)))
+
+
+def w4a4_gemm_rowmax(q_act, scale_act, q_w, scale_w, out, rowmax, stream=None) -> None:
+    """w4a4_gemm, and rowmax[N, ceil(O / 256)] = max |out| per token and
+    256-channel tile (N > 128)."""
+    N, K2 = q_act.shape
+    O = q_w.shape[0]
+    _check(lib.w4a4_gemm_rowmax(_ptr(q_act), _ptr(scale_act), _ptr(q_w), _ptr(scale_w),
+                                int(N), int(2 * K2), int(O), _ptr(out), _ptr(rowmax),
+                                _stream(stream)))
+
+
+def respin_quantize_rowmax(u, rowmax, q_packed, scale, flags: int = 0, stream=None) -> None:
+    """Per-token codes and scales of bf16 u [N, D] from its partial row
+    maxima rowmax [N, D / 256]."""
+    N, D = u.shape
+    _check(lib.respin_quantize_rowmax(_ptr(u), _ptr(rowmax), int(N), int(D), _ptr(q_packed),
+                                      _ptr(scale), ctypes.c_uint(flags), _stream(stream)))
 
 
 def _host_f32(a, shape, name):

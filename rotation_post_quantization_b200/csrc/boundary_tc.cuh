@@ -519,4 +519,39 @@ boundary_quant_rows_kernel(const void* __restrict__ h, int N, int D, uint8_t* __
   }
 }
 
+// Codes and scales of rows of a bf16 matrix u [N, D] whose per-row maxima of
+// |u| come in `parts` partial maxima per row (rowmax [N, parts], e.g. one per
+// 256-column tile from the GEMM that wrote u). Rows are taken from the last
+// to the first, so the rows written last (still in L2) are read first.
+__global__ void __launch_bounds__(256)
+quant_rowmax_kernel(const void* __restrict__ u, const float* __restrict__ rowmax, int N, int D, int parts,
+                    uint8_t* __restrict__ q_out, float* __restrict__ scale_out, float qmax) {
+  constexpr int VPT = 8;
+  const int tid = threadIdx.x;
+  const int nv = D / 8;
+  grid_dep_wait();   // u and its row maxima come from the previous kernel
+  for (int k = blockIdx.x; k < N; k += gridDim.x) {
+    const int row = N - 1 - k;
+    float amax = 0.f;
+    for (int p = 0; p < parts; ++p) amax = fmaxf(amax, rowmax[static_cast<size_t>(row) * parts + p]);
+    float inv, sc;
+    inv_and_scale(amax, qmax, inv, sc);
+    for (int v0 = 0; v0 < nv; v0 += 256 * VPT) {
+      uint4 hv[VPT];
+#pragma unroll
+      for (int j = 0; j < VPT; ++j) {
+        const int v = v0 + tid + 256 * j;
+        hv[j] = make_uint4(0u, 0u, 0u, 0u);
+        if (v < nv) hv[j] = reinterpret_cast<const uint4*>(static_cast<const bf16*>(u) + static_cast<size_t>(row) * D)[v];
+      }
+#pragma unroll
+      for (int j = 0; j < VPT; ++j) {
+        const int v = v0 + tid + 256 * j;
+        if (v < nv) reinterpret_cast<uint32_t*>(q_out + static_cast<size_t>(row) * (D / 2))[v] = quantize8(hv[j], inv);
+      }
+    }
+    if (tid == 0) scale_out[row] = sc;
+  }
+}
+
 }  // namespace respin

@@ -1012,7 +1012,7 @@ static bool make_tmap_out(CUtensorMap* m, void* ptr, uint64_t rows, uint64_t col
 
 static respin_status_t gemm_common(const uint8_t* q_act, const float* scale_act, const uint8_t* q_w,
                                    const float* scale_w, int N, int K, int O, void* out,
-                                   void* stream, bool i32) {
+                                   void* stream, bool i32, float* rowmax = nullptr) {
   t_last_error.clear();
   if (N < 0) return fail(RESPIN_ERR_INVALID_ARG, "N=%d is negative", N);
   if (K < 128 || K > 65536 || K % 128)
@@ -1028,6 +1028,9 @@ static respin_status_t gemm_common(const uint8_t* q_act, const float* scale_act,
   if (fault_at("launch")) return fail(RESPIN_ERR_CUDA, "injected fault at launch");
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (rowmax != nullptr && N <= RESPIN_GEMM_SKINNY_MAX_TOKENS)
+    return fail(RESPIN_ERR_UNSUPPORTED, "row maxima need N > %d (the tensor-memory GEMM)", RESPIN_GEMM_SKINNY_MAX_TOKENS);
+  if (rowmax != nullptr && !aligned(rowmax, 4)) return fail(RESPIN_ERR_ALIGNMENT, "rowmax must be 4-byte aligned");
   if (N <= RESPIN_GEMM_SKINNY_MAX_TOKENS) return gemm_skinny(q_act, scale_act, q_w, scale_w, N, K, O, out, s, i32);
 
   int dev = 0;
@@ -1068,7 +1071,7 @@ static respin_status_t gemm_common(const uint8_t* q_act, const float* scale_act,
   lc.stream = s;
   lc.attrs = attr;
   lc.numAttrs = 2;
-  void* args[] = {&tmA, &tmB, &tmO, const_cast<float**>(&scale_act), const_cast<float**>(&scale_w), &N, &K, &O};
+  void* args[] = {&tmA, &tmB, &tmO, const_cast<float**>(&scale_act), const_cast<float**>(&scale_w), &N, &K, &O, &rowmax};
   e = cudaLaunchKernelExC(&lc, fn, args);
   if (e != cudaSuccess) return cuda_fail(e, "w4a4_gemm_kernel launch");
   e = cudaGetLastError();
@@ -1084,6 +1087,43 @@ respin_status_t w4a4_gemm(const uint8_t* q_act, const float* scale_act, const ui
 respin_status_t w4a4_gemm_i32(const uint8_t* q_act, const uint8_t* q_w, int N, int K, int O,
                               int32_t* acc_out, void* stream) {
   return gemm_common(q_act, nullptr, q_w, nullptr, N, K, O, acc_out, stream, true);
+}
+
+respin_status_t w4a4_gemm_rowmax(const uint8_t* q_act, const float* scale_act, const uint8_t* q_w,
+                                 const float* scale_w, int N, int K, int O, void* out, float* rowmax,
+                                 void* stream) {
+  if (rowmax == nullptr) {
+    t_last_error.clear();
+    return fail(RESPIN_ERR_INVALID_ARG, "rowmax is NULL");
+  }
+  return gemm_common(q_act, scale_act, q_w, scale_w, N, K, O, out, stream, false, rowmax);
+}
+
+respin_status_t respin_quantize_rowmax(const void* u, const float* rowmax, int N, int D, uint8_t* q_packed,
+                                       float* scale, unsigned flags, void* stream) {
+  t_last_error.clear();
+  if (N < 0) return fail(RESPIN_ERR_INVALID_ARG, "N=%d is negative", N);
+  if (D < 256 || D > 65536 || D % 256)
+    return fail(RESPIN_ERR_UNSUPPORTED, "D=%d: need 256 <= D <= 65536 and D %% 256 == 0", D);
+  if (flags & ~RESPIN_ACT_INT3) return fail(RESPIN_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
+  if (N == 0) return ok();
+  if (u == nullptr || rowmax == nullptr || q_packed == nullptr || scale == nullptr)
+    return fail(RESPIN_ERR_INVALID_ARG, "u, rowmax, q_packed and scale must be non-NULL");
+  if (!aligned(u, 16) || !aligned(q_packed, 16)) return fail(RESPIN_ERR_ALIGNMENT, "u and q_packed must be 16-byte aligned");
+  if (!aligned(rowmax, 4) || !aligned(scale, 4)) return fail(RESPIN_ERR_ALIGNMENT, "rowmax and scale must be 4-byte aligned");
+  if (fault_at("launch")) return fail(RESPIN_ERR_CUDA, "injected fault at launch");
+  int dev = 0, sms = 148;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  float qmax = (flags & RESPIN_ACT_INT3) != 0 ? 3.0f : 7.0f;
+  int parts = D / kGemmBN;
+  const int grid = N < sms * 8 ? N : sms * 8;
+  void* args[] = {const_cast<void**>(&u), const_cast<float**>(&rowmax), &N, &D, &parts, &q_packed, &scale, &qmax};
+  e = launch_dependent(reinterpret_cast<const void*>(&quant_rowmax_kernel), grid, 256, 0,
+                       static_cast<cudaStream_t>(stream), args);
+  if (e != cudaSuccess) return cuda_fail(e, "quant_rowmax_kernel launch");
+  return ok();
 }
 
 respin_status_t respin_factors_from_subspace(int D, int r, const float* Q, const float* R_sub, float* U_r,

@@ -127,7 +127,7 @@ template <int CG, bool I32OUT>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const __grid_constant__ CUtensorMap tmO, const float* __restrict__ sa,
-                 const float* __restrict__ sw, int N, int K, int O) {
+                 const float* __restrict__ sw, int N, int K, int O, float* __restrict__ rowmax) {
   using G = GemmCfg<CG>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -209,7 +209,7 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   };
   // One 32-column chunk of accumulators (256 acc each, lane = row `row` of the
   // tile) -> scaled bf16 (or int32) output block at (colb, y) via staging.
-  auto store_chunk = [&](const uint32_t (&v)[32], int colb, int y, float sa_r, const float* swp) {
+  auto store_chunk = [&](const uint32_t (&v)[32], int colb, int y, float sa_r, const float* swp, float& rmax) {
     if constexpr (I32OUT) {
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
@@ -244,6 +244,7 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
           const float f1 =
               __fmul_rn(__fmul_rn(exact_i22_to_f32(static_cast<int32_t>(v[e + 1]) >> 8), sa_r), ws[2 * u + 1]);
           w[u] = pack_bf16x2(f0, f1);
+          rmax = fmaxf(rmax, fmaxf(fabsf(__uint_as_float(w[u] << 16)), fabsf(__uint_as_float(w[u] & 0xFFFF0000u))));
         }
         piece[j] = make_uint4(w[0], w[1], w[2], w[3]);
       }
@@ -406,6 +407,7 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         __syncwarp();
       }
       const uint32_t tbase = tmem + (static_cast<uint32_t>(quad * 32) << 16) + ab * kGemmBN;
+      float rmax = 0.f;   // this row's max |bf16 output| over the tile
 #pragma unroll 1
       for (int cc = 0; cc < kGemmBN / 32; cc += 2) {
         uint32_t v[2][32];
@@ -417,8 +419,13 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         for (int h = 0; h < 2; ++h) {
           const int colb = n0 + (cc + h) * 32;
           if (colb >= O) break;
-          store_chunk(v[h], colb, y, sa_r, sws + (colb - n0));
+          store_chunk(v[h], colb, y, sa_r, sws + (colb - n0), rmax);
         }
+      }
+      // optional per-(row, channel tile) maxima of |out| for a later per-token
+      // quantization of this output (one writer per entry)
+      if constexpr (!I32OUT) {
+        if (rowmax != nullptr && ok && row < N) rowmax[static_cast<size_t>(row) * ((O + kGemmBN - 1) / kGemmBN) + n0 / kGemmBN] = rmax;
       }
       // hand the accumulator buffer back to the MMA warp (of the leader CTA)
       tc_fence_before();

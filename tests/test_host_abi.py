@@ -153,3 +153,26 @@ def test_selftest_limit_validation():
     assert rq.lib.respin_selftest_wait_limit(0, None) == rq.RESPIN_ERR_INVALID_ARG
     assert rq.lib.respin_selftest_wait_limit(2000001, None) == rq.RESPIN_ERR_INVALID_ARG
     assert "limit_us" in rq.last_error()
+
+
+def test_gemm_rowmax_validation():
+    f = rq.lib.w4a4_gemm_rowmax
+    # no rowmax buffer
+    assert f(A16, A16, A16B, A16B, 256, 256, 32, A16, None, None) == rq.RESPIN_ERR_INVALID_ARG
+    # few tokens: the weight-streaming kernel writes no maxima
+    assert f(A16, A16, A16B, A16B, 128, 256, 32, A16, A16, None) == rq.RESPIN_ERR_UNSUPPORTED
+    # misaligned maxima buffer
+    assert f(A16, A16, A16B, A16B, 256, 256, 32, A16, A16 + 2, None) == rq.RESPIN_ERR_ALIGNMENT
+    assert f(A16, A16, A16B, A16B, 256, 100, 32, A16, A16, None) == rq.RESPIN_ERR_UNSUPPORTED
+    assert rq.last_error()
+
+
+def test_quantize_rowmax_validation():
+    f = rq.lib.respin_quantize_rowmax
+    assert f(A16, A16, 4, 300, A16, A16, 0, None) == rq.RESPIN_ERR_UNSUPPORTED      # D % 256
+    assert f(A16, A16, -1, 256, A16, A16, 0, None) == rq.RESPIN_ERR_INVALID_ARG      # N < 0
+    assert f(A16, A16, 0, 256, A16, A16, 0, None) == rq.RESPIN_OK                   # N == 0
+    assert f(None, A16, 4, 256, A16, A16, 0, None) == rq.RESPIN_ERR_INVALID_ARG
+    assert f(MIS, A16, 4, 256, A16, A16, 0, None) == rq.RESPIN_ERR_ALIGNMENT
+    assert f(A16, A16, 4, 256, A16, A16, 8, None) == rq.RESPIN_ERR_INVALID_ARG       # unknown flag
+    assert rq.last_error()
