@@ -108,9 +108,10 @@ struct respin_plan_s {
   const void* quad_fn = nullptr;
   size_t quad_smem = 0;
   int quad_max = 0;              // co-resident 4-CTA clusters
-  // Tensor-core passes for padded ranks 64 / 128 (boundary_tc.cuh): tensor
-  // maps of the plan's U^T [r_pad, D] and V [D, r_pad] (the factor layout of
-  // the shared-memory cluster kernel).
+  // Tensor-core passes (boundary_tc.cuh): tensor maps of U^T [tc_rp, D] and
+  // V [D, tc_rp], the plan's own factors for padded rank 64 / 128 (the layout
+  // of the shared-memory cluster kernel) or a copy padded to 64 (tc_factors)
+  // for rank 16 / 32 plans on the register-factor cluster kernel.
   bool has_tc = false;
   int tc_rp = 0;                          // padded rank of the passes (64 or 128)
   int tc_min_tokens = 0;                  // calls from this many tokens on take them
@@ -124,9 +125,10 @@ struct respin_plan_s {
 
 // Calls with at least this many tokens take the tensor-core passes when the
 // plan has them: padded rank 64 / 128, and padded rank 16 / 32 on the
-// register-factor cluster kernel (D = 8192). Measured on B200 at D = 8192
-// (passes vs cluster kernel): r = 64: 33 vs 34 us at 256 tokens, 159 vs
-// 672 us at 8192; r = 32: 68 vs 62 us at 2048 tokens, 159 vs 222 us at 8192.
+// register-factor cluster kernel (D = 8192). Crossovers measured on B200 at
+// D = 8192 (passes vs cluster kernel, before the passes became dependent
+// launches): r = 64: 33 vs 34 us at 256 tokens; r = 32: 68 vs 62 us at 2048
+// tokens and 159 vs 222 us at 8192 (now 140 us).
 #ifndef RESPIN_TC_MIN_TOKENS
 #define RESPIN_TC_MIN_TOKENS 256
 #endif
