@@ -93,13 +93,13 @@ boundary_tc_project_kernel(const __grid_constant__ CUtensorMap tmR, const __grid
   auto full = [&](int s) { return bars + 8 * s; };
   auto empty = [&](int s) { return bars + 8 * (C::STG + s); };
   const uint32_t done = bars + 16 * C::STG;
-  volatile int* misc = reinterpret_cast<volatile int*>(smem + C::oMisc + 16);   // [0] issued [1] consumed [2] abort
+  volatile int* misc = reinterpret_cast<volatile int*>(smem + C::oMisc + 16);   // [1] consumed [2] abort
   const uint32_t tslot = base + C::oMisc;
 
   if (tid == 0) {
-    for (int s = 0; s < C::STG; ++s) { mbar_init(full(s), 1); mbar_init(empty(s), 1); }
+    for (int s = 0; s < C::STG; ++s) { mbar_init(full(s), 2); mbar_init(empty(s), 1); }   // full: A and B copies
     mbar_init(done, 1);
-    misc[0] = 0; misc[1] = 0; misc[2] = 0;
+    misc[1] = 0; misc[2] = 0;
     fence_mbarrier_init();
     asm volatile("prefetch.tensormap [%0];" ::"l"(&tmR) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(&tmU) : "memory");
@@ -114,18 +114,30 @@ boundary_tc_project_kernel(const __grid_constant__ CUtensorMap tmR, const __grid
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + C::oMisc);
 
-  if (warp == 0 && lane == 0) {
-    // ---- producer: residual and U^T K blocks
-    for (int i = 0; i < nk; ++i) {
+  if (warp == 0 && lane < 2 * C::STG) {
+    // ---- producer lanes: lane 2s copies the residual K blocks of stage s,
+    // lane 2s + 1 the U^T K blocks (copies issued by one thread complete one
+    // after the other, so every stream of copies has its own thread)
+    const int s = lane >> 1;
+    const bool is_u = (lane & 1) != 0;
+    int last = -1;
+    for (int i = s; i < nk; i += C::STG) {
       if (misc[2]) break;
-      const int s = i % C::STG;
-      if (!mbar_wait(empty(s), ((i / C::STG) & 1) ^ 1, kSiteTcFree)) { misc[2] = 1; break; }
+      const int u = i / C::STG;
+      if (!mbar_wait(empty(s), (u & 1) ^ 1, kSiteTcFree)) { misc[2] = 1; break; }
       const uint32_t dst = base + s * C::Stage;
-      mbar_arrive_expect_tx(full(s), C::Stage);
-      tma_load_2d(dst, &tmR, (kb0 + i) * 64, m0, full(s));
-      tma_load_2d(dst + C::ABytes, &tmU, (kb0 + i) * 64, 0, full(s));
-      misc[0] = i + 1;
+      if (is_u) {
+        mbar_arrive_expect_tx(full(s), C::BBytes);
+        tma_load_2d(dst + C::ABytes, &tmU, (kb0 + i) * 64, 0, full(s));
+      } else {
+        mbar_arrive_expect_tx(full(s), C::ABytes);
+        tma_load_2d(dst, &tmR, (kb0 + i) * 64, m0, full(s));
+      }
+      last = u;
     }
+    // after a give-up: the copies this lane issued have landed before the
+    // shared memory is released
+    if (last >= 0) mbar_wait(full(s), last & 1, kSiteTcLoad);
   } else if (warp == 1 && lane == 0) {
     // ---- MMA issuer
     constexpr uint32_t idesc = umma_idesc_bf16(kTcBM, RP);
@@ -144,10 +156,6 @@ boundary_tc_project_kernel(const __grid_constant__ CUtensorMap tmR, const __grid
     tc_commit(done);   // also after a give-up: completes once the issued MMAs have
   }
   __syncthreads();
-  if (tid == 0) {
-    // copies issued but not consumed (only after a give-up)
-    for (int i = misc[1]; i < misc[0]; ++i) mbar_wait(full(i % C::STG), (i / C::STG) & 1, kSiteTcLoad);
-  }
   bool ok = mbar_wait(done, 0, kSiteTcAccum);
   ok = ok && misc[2] == 0 && misc[1] == nk;
   tc_fence_after();
@@ -239,7 +247,7 @@ boundary_tc_reproject_kernel(const __grid_constant__ CUtensorMap tmRc, const __g
 
   if (tid == 0) {
     for (int s = 0; s < C::BST; ++s) { mbar_init(bfull(s), 1); mbar_init(bempty(s), 1); }
-    for (int s = 0; s < C::CST; ++s) { mbar_init(cfull(s), 1); mbar_init(cempty(s), 4); }
+    for (int s = 0; s < C::CST; ++s) { mbar_init(cfull(s), 2); mbar_init(cempty(s), 4); }   // residual + x copies
     for (int a = 0; a < 2; ++a) { mbar_init(afull(a), 1); mbar_init(aempty(a), 8); }
     mbar_init(opa_full, 8);
     mbar_init(opa_empty, 1);
@@ -261,29 +269,33 @@ boundary_tc_reproject_kernel(const __grid_constant__ CUtensorMap tmRc, const __g
   auto new_m = [&](int i) { return i == 0 || tile_m(i) != tile_m(i - 1); };
 
   if (warp == 0) {
-    // ---- producer lanes: lane c < CST owns chunk stage c, lane 16 + s owns
-    // V stage s; each stage has at most one copy in flight. The chunk stages
-    // form two rings, one per epilogue half (stages h HST .. h HST + HST - 1
-    // carry half h's chunks 2h, 2h + 1 of every tile, in order), so every
-    // stage is consumed by the same four warps in order and no consumer can
-    // run two phases ahead of a stage.
+    // ---- producer lanes: lane c < CST copies the residual chunks of stage
+    // c and lane 8 + c its x chunks (copies issued by one thread complete one
+    // after the other), lane 16 + s owns V stage s; each stage has at most
+    // one fill in flight. The chunk stages form two rings, one per epilogue
+    // half (stages h HST .. h HST + HST - 1 carry half h's chunks 2h, 2h + 1
+    // of every tile, in order), so every stage is consumed by the same four
+    // warps in order and no consumer can run two phases ahead of a stage.
+    static_assert(C::CST <= 8, "chunk producer lanes");
     int last = -1;   // this lane's last issued use (for the final drain)
-    if (lane < C::CST) {
-      const int h = lane / C::HST, j = lane % C::HST;
+    if (lane < 16 && (lane & 7) < C::CST) {
+      const int st = lane & 7;
+      const bool is_x = lane >= 8;
+      const int h = st / C::HST, j = st % C::HST;
       const int np = 2 * nloc;   // chunks of half h
       for (int pidx = j; pidx < np; pidx += C::HST) {
         if (*abort_flag) break;
         const int u = pidx / C::HST;
-        if (!mbar_wait(cempty(lane), (u & 1) ^ 1, kSiteTcFree)) { *abort_flag = 1; break; }
+        if (!mbar_wait(cempty(st), (u & 1) ^ 1, kSiteTcFree)) { *abort_flag = 1; break; }
         const int i = pidx >> 1, c = 2 * h + (pidx & 1);
         const int x0 = tile_n(i) * kTcBN + c * kTcChunk, y0 = tile_m(i) * kTcBM;
-        const uint32_t dst = base + C::oC + lane * C::CBytes;
-        mbar_arrive_expect_tx(cfull(lane), C::CBytes);
-        tma_load_2d(dst, &tmRc, x0, y0, cfull(lane));
-        tma_load_2d(dst + C::CHalf, &tmXc, x0, y0, cfull(lane));
+        const uint32_t dst = base + C::oC + st * C::CBytes;
+        mbar_arrive_expect_tx(cfull(st), C::CHalf);
+        if (is_x) tma_load_2d(dst + C::CHalf, &tmXc, x0, y0, cfull(st));
+        else tma_load_2d(dst, &tmRc, x0, y0, cfull(st));
         last = u;
       }
-      if (last >= 0) mbar_wait(cfull(lane), last & 1, kSiteTcLoad);
+      if (last >= 0) mbar_wait(cfull(st), last & 1, kSiteTcLoad);
     } else if (lane >= 16 && lane < 16 + C::BST) {
       const int s = lane - 16;
       for (int i = s; i < nloc; i += C::BST) {
