@@ -932,9 +932,9 @@ respin_status_t respin_boundary_forward(respin_plan_t plan, const void* x, const
 }
 
 extern "C++" {
-template <int CG, bool I32>
+template <int CG, bool I32, bool RM = false>
 const void* gemm_fn() {
-  return reinterpret_cast<const void*>(&w4a4_gemm_kernel<CG, I32>);
+  return reinterpret_cast<const void*>(&w4a4_gemm_kernel<CG, I32, RM>);
 }
 }
 
@@ -954,9 +954,11 @@ static cudaError_t gemm_prepare(int dev, GemmDeviceInfo* info) {
   GemmDeviceInfo& d = infos[dev];
   if (!d.ready) {
     cudaError_t e = cudaSuccess;
-    const void* fns[4] = {gemm_fn<1, false>(), gemm_fn<1, true>(), gemm_fn<2, false>(), gemm_fn<2, true>()};
-    const int smem[4] = {GemmCfg<1>::Smem, GemmCfg<1>::Smem, GemmCfg<2>::Smem, GemmCfg<2>::Smem};
-    for (int i = 0; i < 4 && e == cudaSuccess; ++i)
+    const void* fns[6] = {gemm_fn<1, false>(), gemm_fn<1, true>(), gemm_fn<2, false>(),
+                          gemm_fn<2, true>(), gemm_fn<1, false, true>(), gemm_fn<2, false, true>()};
+    const int smem[6] = {GemmCfg<1>::Smem, GemmCfg<1>::Smem, GemmCfg<2>::Smem,
+                         GemmCfg<2>::Smem, GemmCfg<1>::Smem, GemmCfg<2>::Smem};
+    for (int i = 0; i < 6 && e == cudaSuccess; ++i)
       e = cudaFuncSetAttribute(fns[i], cudaFuncAttributeMaxDynamicSharedMemorySize, smem[i]);
     if (e != cudaSuccess) return e;
     e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
@@ -1053,8 +1055,9 @@ static respin_status_t gemm_common(const uint8_t* q_act, const float* scale_act,
       !make_tmap_u8(&tmB, q_w, O, K / 2, kGemmBN / CG, kGemmBK / 2) ||
       !make_tmap_out(&tmO, out, N, O, i32))
     return fail(RESPIN_ERR_CUDA, "cuTensorMapEncodeTiled failed for the GEMM operands or output");
-  const void* fn = CG == 2 ? (i32 ? gemm_fn<2, true>() : gemm_fn<2, false>())
-                           : (i32 ? gemm_fn<1, true>() : gemm_fn<1, false>());
+  const void* fn = rowmax != nullptr ? (CG == 2 ? gemm_fn<2, false, true>() : gemm_fn<1, false, true>())
+                   : CG == 2         ? (i32 ? gemm_fn<2, true>() : gemm_fn<2, false>())
+                                     : (i32 ? gemm_fn<1, true>() : gemm_fn<1, false>());
   const long long groups = CG == 2 ? (tiles < info.max_pairs ? tiles : info.max_pairs)
                                    : (tiles < info.sms ? tiles : info.sms);
   cudaLaunchConfig_t lc = {};

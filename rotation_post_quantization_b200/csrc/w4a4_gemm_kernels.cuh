@@ -123,7 +123,7 @@ __device__ __forceinline__ uint32_t sw64_offset(int r, int j) {
 // (inner dimension first), no swizzle, out-of-range elements zero filled.
 // tmO: the output [N, O] (bf16, or int32 for I32OUT), box {64 bytes, 32 rows},
 // 64-byte swizzle; the store clips rows >= N and columns >= O.
-template <int CG, bool I32OUT>
+template <int CG, bool I32OUT, bool ROWMAX = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const __grid_constant__ CUtensorMap tmO, const float* __restrict__ sa,
@@ -244,7 +244,8 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
           const float f1 =
               __fmul_rn(__fmul_rn(exact_i22_to_f32(static_cast<int32_t>(v[e + 1]) >> 8), sa_r), ws[2 * u + 1]);
           w[u] = pack_bf16x2(f0, f1);
-          rmax = fmaxf(rmax, fmaxf(fabsf(__uint_as_float(w[u] << 16)), fabsf(__uint_as_float(w[u] & 0xFFFF0000u))));
+          if constexpr (ROWMAX)
+            rmax = fmaxf(rmax, fmaxf(fabsf(__uint_as_float(w[u] << 16)), fabsf(__uint_as_float(w[u] & 0xFFFF0000u))));
         }
         piece[j] = make_uint4(w[0], w[1], w[2], w[3]);
       }
@@ -424,8 +425,8 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       }
       // optional per-(row, channel tile) maxima of |out| for a later per-token
       // quantization of this output (one writer per entry)
-      if constexpr (!I32OUT) {
-        if (rowmax != nullptr && ok && row < N) rowmax[static_cast<size_t>(row) * ((O + kGemmBN - 1) / kGemmBN) + n0 / kGemmBN] = rmax;
+      if constexpr (ROWMAX && !I32OUT) {
+        if (ok && row < N) rowmax[static_cast<size_t>(row) * ((O + kGemmBN - 1) / kGemmBN) + n0 / kGemmBN] = rmax;
       }
       // hand the accumulator buffer back to the MMA warp (of the leader CTA)
       tc_fence_before();
