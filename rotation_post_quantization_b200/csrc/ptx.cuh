@@ -403,6 +403,19 @@ __device__ __forceinline__ void tc_mma_i8_pair(uint32_t d_tmem, uint64_t adesc, 
       : "memory");
 }
 
+// The same pair MMA with A read from tensor memory: each CTA holds its 128 A
+// rows in TMEM lanes 0..127 at column address `a_tmem` (K-major, four 8-bit
+// elements per 32-bit column); B comes from shared memory as above.
+__device__ __forceinline__ void tc_mma_i8_pair_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                                  uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::i8 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrive on the barrier at offset `bar` in every CTA of `mask` once all
 // tcgen05 operations issued so far by this thread (over the pair) completed.
 __device__ __forceinline__ void tc_commit_pair_multicast(uint32_t bar, uint16_t mask) {
@@ -469,6 +482,21 @@ __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&v)
 
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// 32 lanes x 16 consecutive 32-bit columns: thread t writes lane (base+t).
+__device__ __forceinline__ void tmem_st_32x32b_x16(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+      : "memory");
+}
+
+// Wait until this thread's earlier tcgen05.st have completed.
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
 // Shared-memory matrix descriptor (tcgen05 format) for a K-major operand in

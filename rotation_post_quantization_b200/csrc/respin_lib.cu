@@ -936,7 +936,27 @@ template <int CG, bool I32, bool RM = false>
 const void* gemm_fn() {
   return reinterpret_cast<const void*>(&w4a4_gemm_kernel<CG, I32, RM>);
 }
+template <bool I32, bool RM = false>
+const void* gemm_ta_fn() {
+  return reinterpret_cast<const void*>(&w4a4_gemm_ta_kernel<I32, RM>);
 }
+}
+
+// CTA pairs read the activation operand from tensor memory
+// (w4a4_gemm_ta_kernel); RESPIN_GEMM_PAIR_SMEM_A=1 builds the pair path on
+// w4a4_gemm_kernel<2, ...> (both operands through shared memory) instead.
+#ifndef RESPIN_GEMM_PAIR_SMEM_A
+#define RESPIN_GEMM_PAIR_SMEM_A 0
+#endif
+static const void* gemm_pair_fn(bool i32, bool rm) {
+#if RESPIN_GEMM_PAIR_SMEM_A
+  return rm ? gemm_fn<2, false, true>() : i32 ? gemm_fn<2, true>() : gemm_fn<2, false>();
+#else
+  return rm ? gemm_ta_fn<false, true>() : i32 ? gemm_ta_fn<true>() : gemm_ta_fn<false>();
+#endif
+}
+static constexpr int kGemmPairThreads = RESPIN_GEMM_PAIR_SMEM_A ? kGemmThreads : kTaThreads;
+static constexpr int kGemmPairSmem = RESPIN_GEMM_PAIR_SMEM_A ? GemmCfg<2>::Smem : GemmTaCfg::Smem;
 
 // The GEMM kernels need the large dynamic shared-memory carve-out; set it
 // once per device and record how many CTA pairs can be co-resident.
@@ -954,10 +974,10 @@ static cudaError_t gemm_prepare(int dev, GemmDeviceInfo* info) {
   GemmDeviceInfo& d = infos[dev];
   if (!d.ready) {
     cudaError_t e = cudaSuccess;
-    const void* fns[6] = {gemm_fn<1, false>(), gemm_fn<1, true>(), gemm_fn<2, false>(),
-                          gemm_fn<2, true>(), gemm_fn<1, false, true>(), gemm_fn<2, false, true>()};
-    const int smem[6] = {GemmCfg<1>::Smem, GemmCfg<1>::Smem, GemmCfg<2>::Smem,
-                         GemmCfg<2>::Smem, GemmCfg<1>::Smem, GemmCfg<2>::Smem};
+    const void* fns[6] = {gemm_fn<1, false>(), gemm_fn<1, true>(),   gemm_pair_fn(false, false),
+                          gemm_pair_fn(true, false), gemm_fn<1, false, true>(), gemm_pair_fn(false, true)};
+    const int smem[6] = {GemmCfg<1>::Smem, GemmCfg<1>::Smem, kGemmPairSmem,
+                         kGemmPairSmem,    GemmCfg<1>::Smem, kGemmPairSmem};
     for (int i = 0; i < 6 && e == cudaSuccess; ++i)
       e = cudaFuncSetAttribute(fns[i], cudaFuncAttributeMaxDynamicSharedMemorySize, smem[i]);
     if (e != cudaSuccess) return e;
@@ -970,8 +990,8 @@ static cudaError_t gemm_prepare(int dev, GemmDeviceInfo* info) {
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     lc.gridDim = dim3(2, 1, 1);
-    lc.blockDim = dim3(kGemmThreads, 1, 1);
-    lc.dynamicSmemBytes = GemmCfg<2>::Smem;
+    lc.blockDim = dim3(kGemmPairThreads, 1, 1);
+    lc.dynamicSmemBytes = kGemmPairSmem;
     lc.attrs = attr;
     lc.numAttrs = 1;
     if (cudaOccupancyMaxActiveClusters(&d.max_pairs, fns[2], &lc) != cudaSuccess) {
@@ -985,9 +1005,10 @@ static cudaError_t gemm_prepare(int dev, GemmDeviceInfo* info) {
 }
 
 // 2-D uint8 tensor map over a row-major [rows, cols] byte matrix with a box
-// of [box_rows, box_cols] (no swizzle, out-of-range reads return zeros).
+// of [box_rows, box_cols] (out-of-range reads return zeros).
 static bool make_tmap_u8(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols,
-                         uint32_t box_rows, uint32_t box_cols) {
+                         uint32_t box_rows, uint32_t box_cols,
+                         CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_NONE) {
   EncodeTiledFn fn = encode_tiled();
   if (!fn) return false;
   const cuuint64_t dims[2] = {cols, rows};
@@ -995,7 +1016,7 @@ static bool make_tmap_u8(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_
   const cuuint32_t box[2] = {box_cols, box_rows};
   const cuuint32_t estr[2] = {1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
             CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -1051,13 +1072,16 @@ static respin_status_t gemm_common(const uint8_t* q_act, const float* scale_act,
   const long long tiles = static_cast<long long>((O + kGemmBN - 1) / kGemmBN) *
                           ((N + kGemmBM * CG - 1) / (kGemmBM * CG));
   CUtensorMap tmA, tmB, tmO;
-  if (!make_tmap_u8(&tmA, q_act, N, K / 2, kGemmBM, kGemmBK / 2) ||
+  // the tensor-memory A path reads packed A rows one per lane: 64-byte swizzle
+  const CUtensorMapSwizzle a_swizzle =
+      (CG == 2 && !RESPIN_GEMM_PAIR_SMEM_A) ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE;
+  if (!make_tmap_u8(&tmA, q_act, N, K / 2, kGemmBM, kGemmBK / 2, a_swizzle) ||
       !make_tmap_u8(&tmB, q_w, O, K / 2, kGemmBN / CG, kGemmBK / 2) ||
       !make_tmap_out(&tmO, out, N, O, i32))
     return fail(RESPIN_ERR_CUDA, "cuTensorMapEncodeTiled failed for the GEMM operands or output");
-  const void* fn = rowmax != nullptr ? (CG == 2 ? gemm_fn<2, false, true>() : gemm_fn<1, false, true>())
-                   : CG == 2         ? (i32 ? gemm_fn<2, true>() : gemm_fn<2, false>())
-                                     : (i32 ? gemm_fn<1, true>() : gemm_fn<1, false>());
+  const void* fn = CG == 2             ? gemm_pair_fn(i32, rowmax != nullptr)
+                   : rowmax != nullptr ? gemm_fn<1, false, true>()
+                                       : (i32 ? gemm_fn<1, true>() : gemm_fn<1, false>());
   const long long groups = CG == 2 ? (tiles < info.max_pairs ? tiles : info.max_pairs)
                                    : (tiles < info.sms ? tiles : info.sms);
   cudaLaunchConfig_t lc = {};
@@ -1071,8 +1095,8 @@ static respin_status_t gemm_common(const uint8_t* q_act, const float* scale_act,
   attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   lc.gridDim = dim3(static_cast<unsigned>(groups * CG), 1, 1);
-  lc.blockDim = dim3(kGemmThreads, 1, 1);
-  lc.dynamicSmemBytes = CG == 2 ? GemmCfg<2>::Smem : GemmCfg<1>::Smem;
+  lc.blockDim = dim3(CG == 2 ? kGemmPairThreads : kGemmThreads, 1, 1);
+  lc.dynamicSmemBytes = CG == 2 ? kGemmPairSmem : GemmCfg<1>::Smem;
   lc.stream = s;
   lc.attrs = attr;
   lc.numAttrs = 2;

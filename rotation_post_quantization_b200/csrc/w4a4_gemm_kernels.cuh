@@ -119,6 +119,97 @@ __device__ __forceinline__ uint32_t sw64_offset(int r, int j) {
   return static_cast<uint32_t>(r * 64 + ((j ^ ((r >> 1) & 3)) << 4));
 }
 
+// Output path of one epilogue warp: a 32-column chunk of accumulators (lane =
+// one token row; 256 acc each) is scaled to bf16 (or shifted back to int32),
+// written into one of EB 32 x 64-byte staging units in shared memory
+// (tensor-map 64-byte swizzle, conflict-free row-per-lane writes), and lane 0
+// sends the unit to global memory with one 2-D tensor store, so every output
+// row segment reaches L2 as whole sectors. int32 output takes two units
+// (16 columns each) per chunk.
+template <bool I32OUT, bool ROWMAX, int EB>
+struct GemmOut {
+  static constexpr int Unit = 32 * 64;
+  const CUtensorMap* tmO;
+  uint8_t* smem;     // generic pointer to shared address `base`
+  uint32_t base;
+  uint32_t ubase;    // this warp's first staging unit (shared address)
+  int lane, O;
+  int unit;
+
+  __device__ __forceinline__ GemmOut(const CUtensorMap* tm, uint8_t* sm, uint32_t b, uint32_t ub, int ln, int o)
+      : tmO(tm), smem(sm), base(b), ubase(ub), lane(ln), O(o), unit(0) {}
+
+  // Staging of one unit: begin() waits until the unit's previous tensor store
+  // has read it and returns its generic address; the caller writes the
+  // lane's four 16-byte pieces (put), then end() sends the unit.
+  __device__ __forceinline__ uint8_t* begin() {
+    if (lane == 0) bulk_wait_group_read<EB - 1>();   // this unit's previous store read it
+    __syncwarp();
+    return smem + (ubase + static_cast<uint32_t>((unit % EB) * Unit) - base);
+  }
+  __device__ __forceinline__ void put(uint8_t* up, int j, uint4 piece) {
+    *reinterpret_cast<uint4*>(up + sw64_offset(lane, j)) = piece;
+  }
+  __device__ __forceinline__ void end(int x, int y) {
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_2d(tmO, x, y, ubase + static_cast<uint32_t>((unit % EB) * Unit));
+      bulk_commit_group();
+    }
+    ++unit;
+  }
+
+  // chunk v (columns colb..colb+31 of row y + lane) with row scale sa_r and
+  // the chunk's 32 channel scales at swp; rmax takes the max |bf16 output|.
+  // Each 16-byte piece goes to shared memory as soon as it is formed.
+  __device__ __forceinline__ void chunk(const uint32_t (&v)[32], int colb, int y, float sa_r, const float* swp,
+                                        float& rmax) {
+    if constexpr (I32OUT) {
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        if (colb + 16 * half >= O) break;
+        uint8_t* up = begin();
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int e = 16 * half + 4 * j;
+          put(up, j,
+              make_uint4(static_cast<uint32_t>(static_cast<int32_t>(v[e]) >> 8),
+                         static_cast<uint32_t>(static_cast<int32_t>(v[e + 1]) >> 8),
+                         static_cast<uint32_t>(static_cast<int32_t>(v[e + 2]) >> 8),
+                         static_cast<uint32_t>(static_cast<int32_t>(v[e + 3]) >> 8)));
+        }
+        end(colb + 16 * half, y);
+      }
+    } else {
+      uint8_t* up = begin();
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (colb + 8 * j >= O) {   // O % 16 == 0: a chunk is full or half full
+          put(up, j, make_uint4(0u, 0u, 0u, 0u));
+          continue;
+        }
+        const float4 w0 = reinterpret_cast<const float4*>(swp)[2 * j];
+        const float4 w1 = reinterpret_cast<const float4*>(swp)[2 * j + 1];
+        const float ws[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+        uint32_t w[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int e = 8 * j + 2 * u;
+          const float f0 = __fmul_rn(__fmul_rn(exact_i22_to_f32(static_cast<int32_t>(v[e]) >> 8), sa_r), ws[2 * u]);
+          const float f1 =
+              __fmul_rn(__fmul_rn(exact_i22_to_f32(static_cast<int32_t>(v[e + 1]) >> 8), sa_r), ws[2 * u + 1]);
+          w[u] = pack_bf16x2(f0, f1);
+          if constexpr (ROWMAX)
+            rmax = fmaxf(rmax, fmaxf(fabsf(__uint_as_float(w[u] << 16)), fabsf(__uint_as_float(w[u] & 0xFFFF0000u))));
+        }
+        put(up, j, make_uint4(w[0], w[1], w[2], w[3]));
+      }
+      end(colb, y);
+    }
+  }
+};
+
 // tmA: uint8 [N, K/2] box {64, 128}; tmB: uint8 [O, K/2] box {64, 256/CG}
 // (inner dimension first), no swizzle, out-of-range elements zero filled.
 // tmO: the output [N, O] (bf16, or int32 for I32OUT), box {64 bytes, 32 rows},
@@ -190,68 +281,8 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   // Epilogue output staging (epilogue warps): EB 32 x 64-byte units per warp,
   // each written to global memory by one tensor store.
   const int quad = warp & 3;   // hardware rule: warp w reads TMEM lanes 32*(w%4)..
-  const uint32_t ubase = ebase + static_cast<uint32_t>(quad * G::EB * G::Unit);
-  int unit = 0;
-  auto stage_unit = [&](const uint4 (&piece)[4], int x, int y) {
-    if (lane == 0) bulk_wait_group_read<G::EB - 1>();   // this unit's previous store read it
-    __syncwarp();
-    const uint32_t u = ubase + static_cast<uint32_t>((unit % G::EB) * G::Unit);
-    uint8_t* up = smem + (u - base);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) *reinterpret_cast<uint4*>(up + sw64_offset(lane, j)) = piece[j];
-    fence_proxy_async_smem();
-    __syncwarp();
-    if (lane == 0) {
-      tma_store_2d(&tmO, x, y, u);
-      bulk_commit_group();
-    }
-    ++unit;
-  };
-  // One 32-column chunk of accumulators (256 acc each, lane = row `row` of the
-  // tile) -> scaled bf16 (or int32) output block at (colb, y) via staging.
-  auto store_chunk = [&](const uint32_t (&v)[32], int colb, int y, float sa_r, const float* swp, float& rmax) {
-    if constexpr (I32OUT) {
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        if (colb + 16 * half >= O) break;
-        uint4 piece[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int e = 16 * half + 4 * j;
-          piece[j] = make_uint4(static_cast<uint32_t>(static_cast<int32_t>(v[e]) >> 8),
-                                static_cast<uint32_t>(static_cast<int32_t>(v[e + 1]) >> 8),
-                                static_cast<uint32_t>(static_cast<int32_t>(v[e + 2]) >> 8),
-                                static_cast<uint32_t>(static_cast<int32_t>(v[e + 3]) >> 8));
-        }
-        stage_unit(piece, colb + 16 * half, y);
-      }
-    } else {
-      uint4 piece[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        if (colb + 8 * j >= O) {   // O % 16 == 0: a chunk is full or half full
-          piece[j] = make_uint4(0u, 0u, 0u, 0u);
-          continue;
-        }
-        const float4 w0 = reinterpret_cast<const float4*>(swp)[2 * j];
-        const float4 w1 = reinterpret_cast<const float4*>(swp)[2 * j + 1];
-        const float ws[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-        uint32_t w[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int e = 8 * j + 2 * u;
-          const float f0 = __fmul_rn(__fmul_rn(exact_i22_to_f32(static_cast<int32_t>(v[e]) >> 8), sa_r), ws[2 * u]);
-          const float f1 =
-              __fmul_rn(__fmul_rn(exact_i22_to_f32(static_cast<int32_t>(v[e + 1]) >> 8), sa_r), ws[2 * u + 1]);
-          w[u] = pack_bf16x2(f0, f1);
-          if constexpr (ROWMAX)
-            rmax = fmaxf(rmax, fmaxf(fabsf(__uint_as_float(w[u] << 16)), fabsf(__uint_as_float(w[u] & 0xFFFF0000u))));
-        }
-        piece[j] = make_uint4(w[0], w[1], w[2], w[3]);
-      }
-      stage_unit(piece, colb, y);
-    }
-  };
+  GemmOut<I32OUT, ROWMAX, G::EB> out(&tmO, smem, base, ebase + static_cast<uint32_t>(quad * G::EB * G::Unit),
+                                     lane, O);
 
   if (warp < kGemmProducerWarps) {
     // ------------------------------------------------ producers: widen packed -> int8
@@ -420,7 +451,7 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         for (int h = 0; h < 2; ++h) {
           const int colb = n0 + (cc + h) * 32;
           if (colb >= O) break;
-          store_chunk(v[h], colb, y, sa_r, sws + (colb - n0), rmax);
+          out.chunk(v[h], colb, y, sa_r, sws + (colb - n0), rmax);
         }
       }
       // optional per-(row, channel tile) maxima of |out| for a later per-token
@@ -448,6 +479,334 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     tc_fence_after();
     if constexpr (CG == 2) tmem_dealloc_pair(tmem, 512);
     else tmem_dealloc(tmem, 512);
+  }
+}
+
+
+// ---------------------------------------------------------------------------
+// CTA-pair GEMM with the activation operand in tensor memory.
+//
+// In the kernel above both widened operands pass through shared memory. Here
+// the producers widen A straight into tensor memory (tcgen05.st, one token
+// row per lane) and the MMA reads A from there (tcgen05.mma with A in TMEM):
+// a stage's shared memory holds only the widened B (16 KB instead of 32 KB),
+// the A write and read leave the shared-memory pipe, and the space freed
+// buys a deeper packed ring (7 stages): under load a packed copy takes
+// 1-2.5 us from issue to arrival (per-K-block timestamps), which 4 stages did
+// not cover (8192 x 8192 -> 28672: 1514 us with both operands in shared
+// memory and 4 packed stages, 1209 us here).
+//
+// Tensor memory (512 columns): the int32 accumulator of the current tile in
+// columns [0, 256) (one buffer), then US A stages of 32 columns (128 int8 K
+// values per row, four per 32-bit column). With one accumulator the next
+// tile's first MMA waits until the epilogues have read the accumulator, so
+// 16 epilogue warps (four per TMEM lane quarter, 64 columns each) read their
+// whole share in one round and hand it back before converting anything
+// (measured with 8 warps that converted half their columns first: the
+// tensor pipe idled ~1.4 us at every tile switch). Splitting the hand-over
+// by column halves instead needs N = 128 MMAs, which measured 40 % slower
+// than N = 256.
+//
+// Warps: 0-3 producers (warp w widens the A rows of TMEM lane quarter w and
+// four 16-byte B chunks per thread), 4 MMA (leader CTA, one thread), 5-20
+// epilogue, 21 TMA.
+constexpr int kTaProducerWarps = 4;
+constexpr int kTaMmaWarp = 4;
+constexpr int kTaEpiWarp0 = 5;
+constexpr int kTaEpilogueWarps = 16;
+constexpr int kTaTmaWarp = kTaEpiWarp0 + kTaEpilogueWarps;   // 21
+constexpr int kTaThreads = (kTaTmaWarp + 1) * 32;            // 704
+
+#ifndef RESPIN_GEMM_TA_US
+#define RESPIN_GEMM_TA_US 4
+#endif
+#ifndef RESPIN_GEMM_TA_PS
+#define RESPIN_GEMM_TA_PS 7
+#endif
+#ifndef RESPIN_GEMM_TA_EB
+#define RESPIN_GEMM_TA_EB 1
+#endif
+
+struct GemmTaCfg {
+  static constexpr int BNC = kGemmBN / 2;                       // channel rows staged by this CTA
+  static constexpr int US = RESPIN_GEMM_TA_US;                  // widened stages (B in smem, A in TMEM)
+  static constexpr int PS = RESPIN_GEMM_TA_PS;                  // packed stages
+  static constexpr int AC = kGemmBK / 32;                       // packed 16-byte A pieces per row
+  static constexpr int BStage = BNC * kGemmBK;                  // widened B bytes
+  static constexpr int PAStage = kGemmBM * kGemmBK / 2;         // packed A bytes
+  static constexpr int PStage = (kGemmBM + BNC) * kGemmBK / 2;  // packed A + B bytes
+  static constexpr int BChunksPerThread = BNC * (kGemmBK / 32) / (kTaProducerWarps * 32);
+  static constexpr int TileM = 2 * kGemmBM;
+  static constexpr int EB = RESPIN_GEMM_TA_EB;                  // output staging units per epilogue warp
+  static constexpr int Unit = 32 * 64;
+  static constexpr int EpiCols = kGemmBN / 4;                   // accumulator columns per epilogue warp
+  static constexpr int SwBytes = EpiCols * 4;
+  static constexpr int AccCols = kGemmBN;                       // TMEM columns of the accumulator
+  static constexpr int ACols = kGemmBK / 4;                     // TMEM columns per A stage
+  static constexpr int RmaxBytes = 2 * 4 * 4 * 32 * 4;          // [2][quarter][part][row] partial row maxima
+  static constexpr int Smem = US * BStage + PS * PStage + kTaEpilogueWarps * (EB * Unit + SwBytes) +
+                              RmaxBytes + 1024 + 256;
+  static_assert(AccCols + US * ACols <= 512, "TMEM: accumulator and A stages");
+  static_assert(2 * PS <= 32, "one issuing lane pair per packed stage");
+  static_assert(BChunksPerThread * kTaProducerWarps * 32 == BNC * (kGemmBK / 32), "chunk split");
+  static_assert(kTaProducerWarps == 4, "producer warp w widens the A rows of TMEM lane quarter w");
+  static_assert(8 * (2 * US + 2 * PS + 2) + 4 <= 256, "barrier area");
+};
+
+// tmA: uint8 [N, K/2] box {64, 128}, 64-byte swizzle (row r's 16-byte piece j
+// lands at r*64 + ((j ^ ((r >> 1) & 3)) << 4): the eight rows a quarter-warp
+// reads fall in eight distinct bank groups); tmB: uint8 [O, K/2] box
+// {64, 128}, no swizzle; tmO as above. Launched as clusters of 2.
+template <bool I32OUT, bool ROWMAX = false>
+__global__ void __launch_bounds__(kTaThreads, 1)
+w4a4_gemm_ta_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                    const __grid_constant__ CUtensorMap tmO, const float* __restrict__ sa,
+                    const float* __restrict__ sw, int N, int K, int O, float* __restrict__ rowmax) {
+  using G = GemmTaCfg;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (base - raw);
+  const uint32_t pbase = base + G::US * G::BStage;    // packed ring
+  const uint32_t ebase = pbase + G::PS * G::PStage;   // output staging units
+  const uint32_t swbase = ebase + kTaEpilogueWarps * G::EB * G::Unit;   // channel scales
+  const uint32_t rmbase = swbase + kTaEpilogueWarps * G::SwBytes;       // partial row maxima
+  const uint32_t bars = rmbase + G::RmaxBytes;
+  const uint32_t full0 = bars;                      // [US] widened stage ready (leader counts both CTAs)
+  const uint32_t empty0 = full0 + 8 * G::US;        // [US] widened stage consumed (MMA commit)
+  const uint32_t pfull0 = empty0 + 8 * G::US;       // [PS] packed stage landed (TMA)
+  const uint32_t pempty0 = pfull0 + 8 * G::PS;      // [PS] packed stage consumed
+  const uint32_t afull = pempty0 + 8 * G::PS;       // accumulator complete (MMA commit)
+  const uint32_t aempty = afull + 8;                // accumulator read out (leader)
+  const uint32_t tslot = aempty + 8;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int group = static_cast<int>(blockIdx.x) / 2;
+  const int ngroups = static_cast<int>(gridDim.x) / 2;
+  const int KB = K / kGemmBK;
+  const int mtiles = (N + G::TileM - 1) / G::TileM;
+  const int ntiles = (O + kGemmBN - 1) / kGemmBN;
+  const int tiles = mtiles * ntiles;
+
+  if (tid == 0) {
+    for (int s = 0; s < G::US; ++s) {
+      mbar_init(full0 + 8 * s, 2 * kTaProducerWarps);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    for (int s = 0; s < G::PS; ++s) {
+      mbar_init(pfull0 + 8 * s, 2);   // the A and the B copy each arrive with their bytes
+      mbar_init(pempty0 + 8 * s, kTaProducerWarps);
+    }
+    mbar_init(afull, 1);
+    mbar_init(aempty, 2 * kTaEpilogueWarps);
+    fence_mbarrier_init();
+  }
+  if (warp == 0) {
+    tmem_alloc_pair(tslot, 512);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync();
+  tc_fence_after();
+  grid_dep_launch();   // the next kernel of the stream may be scheduled
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + (tslot - base));
+  const uint32_t full_leader0 = map_to_rank(full0, 0);
+  const uint32_t aempty_leader = map_to_rank(aempty, 0);
+
+  if (warp < kTaProducerWarps) {
+    // ------------------------------------------------ producers: widen packed -> int8
+    const int quad = warp;       // TMEM lanes 32*quad.. (hardware rule: warp w, lanes 32*(w%4)..)
+    const int arow = quad * 32 + lane;
+    const uint32_t a_lane = tmem + (static_cast<uint32_t>(quad * 32) << 16) + G::AccCols;
+    bool ok = true;
+    int kstep = 0;
+    for (int t = group; t < tiles; t += ngroups) {
+      for (int kb = 0; kb < KB; ++kb, ++kstep) {
+        const int ps = kstep % G::PS, s = kstep % G::US;
+        if (ok) ok = mbar_wait(pfull0 + 8 * ps, (kstep / G::PS) & 1, kSiteGemmPackedFull);
+        const uint8_t* pk = smem + (pbase - base) + ps * G::PStage;
+        uint4 a[G::AC], b[G::BChunksPerThread];
+#pragma unroll
+        for (int j = 0; j < G::AC; ++j)
+          a[j] = *reinterpret_cast<const uint4*>(pk + arow * 64 + ((j ^ ((arow >> 1) & 3)) << 4));
+#pragma unroll
+        for (int j = 0; j < G::BChunksPerThread; ++j)   // chunk q = row*4 + c, 16 bytes each
+          b[j] = *reinterpret_cast<const uint4*>(pk + G::PAStage + (tid + j * kTaProducerWarps * 32) * 16);
+        if (ok) ok = mbar_wait(empty0 + 8 * s, ((kstep / G::US) & 1) ^ 1, kSiteGemmEmpty);
+        tc_fence_after();   // the MMAs that read this stage's A columns are complete
+        // B: widened into the 128-byte-swizzled K-major layout
+        uint8_t* sB = smem + s * G::BStage;
+#pragma unroll
+        for (int j = 0; j < G::BChunksPerThread; ++j) {
+          const int q = tid + j * kTaProducerWarps * 32;
+          const int row = q >> 2, c = q & 3;
+          uint8_t* rowp = sB + (row >> 3) * 1024 + (row & 7) * 128;
+          const uint4 p = b[j];
+          const uint4 lo = make_uint4((p.x << 4) & 0xF0F0F0F0u, (p.y << 4) & 0xF0F0F0F0u,
+                                      (p.z << 4) & 0xF0F0F0F0u, (p.w << 4) & 0xF0F0F0F0u);
+          const uint4 hi = make_uint4(p.x & 0xF0F0F0F0u, p.y & 0xF0F0F0F0u, p.z & 0xF0F0F0F0u,
+                                      p.w & 0xF0F0F0F0u);
+          *reinterpret_cast<uint4*>(rowp + (((2 * c) ^ (row & 7)) << 4)) = lo;
+          *reinterpret_cast<uint4*>(rowp + (((2 * c + 1) ^ (row & 7)) << 4)) = hi;
+        }
+        // A: the same K permutation (even codes of a 16-byte piece, then its
+        // odd codes), as 32-bit TMEM columns of this lane's row
+#pragma unroll
+        for (int h = 0; h < G::AC / 2; ++h) {
+          uint32_t w[16];
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            const uint4 p = a[2 * h + j];
+            w[8 * j + 0] = (p.x << 4) & 0xF0F0F0F0u;
+            w[8 * j + 1] = (p.y << 4) & 0xF0F0F0F0u;
+            w[8 * j + 2] = (p.z << 4) & 0xF0F0F0F0u;
+            w[8 * j + 3] = (p.w << 4) & 0xF0F0F0F0u;
+            w[8 * j + 4] = p.x & 0xF0F0F0F0u;
+            w[8 * j + 5] = p.y & 0xF0F0F0F0u;
+            w[8 * j + 6] = p.z & 0xF0F0F0F0u;
+            w[8 * j + 7] = p.w & 0xF0F0F0F0u;
+          }
+          tmem_st_32x32b_x16(a_lane + static_cast<uint32_t>(s * G::ACols + 16 * h), w);
+        }
+        tmem_wait_st();
+        // Stage -> MMA: the TMEM stores are complete and ordered before the
+        // arrival (tcgen05 fence), the shared-memory stores are made visible
+        // to the async proxy; the packed stage is released by the same
+        // proxy fence (its generic reads before the next tensor copy).
+        tc_fence_before();
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive_cluster(full_leader0 + 8 * s);
+          mbar_arrive(pempty0 + 8 * ps);
+        }
+      }
+    }
+  } else if (warp == kTaTmaWarp) {
+    // ------------------------------------------------ TMA warp: packed K blocks
+    grid_dep_wait();   // the codes (and possibly the weights) come from earlier kernels
+    if (lane < 2 * G::PS) {
+      const int stage = lane >> 1;
+      const bool is_b = (lane & 1) != 0;
+      const uint32_t bytes = is_b ? G::PStage - G::PAStage : G::PAStage;
+      bool ok = true;
+      int kstep = 0;
+      for (int t = group; t < tiles; t += ngroups) {
+        const int arow = (t / ntiles) * G::TileM + static_cast<int>(rank) * kGemmBM;
+        const int brow = (t % ntiles) * kGemmBN + static_cast<int>(rank) * G::BNC;
+        for (int kb = 0; kb < KB; ++kb, ++kstep) {
+          const int ps = kstep % G::PS;
+          if (ps != stage) continue;
+          if (ok) ok = mbar_wait(pempty0 + 8 * ps, ((kstep / G::PS) & 1) ^ 1, kSiteGemmPackedEmpty);
+          if (!ok) continue;
+          const uint32_t dst = pbase + ps * G::PStage;
+          mbar_arrive_expect_tx(pfull0 + 8 * ps, bytes);
+          if (is_b) tma_load_2d(dst + G::PAStage, &tmB, kb * (kGemmBK / 2), brow, pfull0 + 8 * ps);
+          else tma_load_2d(dst, &tmA, kb * (kGemmBK / 2), arow, pfull0 + 8 * ps);
+        }
+      }
+    }
+  } else if (warp == kTaMmaWarp) {
+    // ------------------------------------------------ MMA issuer (leader CTA)
+    if (rank == 0) {
+      constexpr uint32_t idesc = umma_idesc_s8(G::TileM, kGemmBN);
+      bool ok = true;
+      int kstep = 0, local = 0;
+      for (int t = group; t < tiles; t += ngroups, ++local) {
+        // both CTAs' epilogues have read the previous tile's accumulator
+        if (ok) ok = mbar_wait_cluster(aempty, (local & 1) ^ 1, kSiteGemmAccum);
+        tc_fence_after();
+        for (int kb = 0; kb < KB; ++kb, ++kstep) {
+          const int s = kstep % G::US;
+          if (ok) ok = mbar_wait_cluster(full0 + 8 * s, (kstep / G::US) & 1, kSiteGemmFull);
+          tc_fence_after();
+          if (lane == 0 && ok) {
+            const uint32_t b_addr = base + s * G::BStage;
+            const uint32_t a_tm = tmem + G::AccCols + static_cast<uint32_t>(s * G::ACols);
+#pragma unroll
+            for (int k = 0; k < kGemmBK / 32; ++k) {
+              const uint64_t bd = umma_desc_sw128(b_addr + 32 * k);
+              tc_mma_i8_pair_ta(tmem, a_tm + 8 * k, bd, idesc, (kb | k) != 0 ? 1u : 0u);
+            }
+            tc_commit_pair_multicast(empty0 + 8 * s, 0x3);
+          }
+          __syncwarp();
+        }
+        if (lane == 0) tc_commit_pair_multicast(afull, 0x3);
+        __syncwarp();
+      }
+    }
+  } else {
+    // ------------------------------------------------ epilogue warps
+    // Four warps per TMEM lane quarter, 64 accumulator columns each: a warp
+    // holds its whole share in registers after one round of tcgen05.ld, so
+    // the accumulator goes back to the MMA warp before any conversion.
+    const int e = warp - kTaEpiWarp0;
+    const int quad = warp & 3;   // TMEM lanes 32*quad.. = token rows of this warp
+    const int part = e >> 2;     // accumulator columns [64 part, 64 part + 64)
+    GemmOut<I32OUT, ROWMAX, G::EB> out(&tmO, smem, base, ebase + static_cast<uint32_t>(e * G::EB * G::Unit), lane, O);
+    float* sws = reinterpret_cast<float*>(smem + (swbase - base) + e * G::SwBytes);
+    float* rmx = reinterpret_cast<float*>(smem + (rmbase - base));
+    grid_dep_wait();   // the activation scales and the output buffer
+    bool ok = true;
+    int local = 0;
+    for (int t = group; t < tiles; t += ngroups, ++local) {
+      const int m0 = (t / ntiles) * G::TileM + static_cast<int>(rank) * kGemmBM;
+      const int n0 = (t % ntiles) * kGemmBN;
+      const int c0 = n0 + part * G::EpiCols;   // first output column of this warp
+      const int y = m0 + quad * 32;            // first row of this warp's blocks
+      const int row = y + lane;
+      float sa_r = 0.f;
+      float2 sw2 = make_float2(0.f, 0.f);
+      if constexpr (!I32OUT) {
+        if (row < N) sa_r = __ldg(sa + row);
+        if (c0 + 2 * lane < O) sw2 = __ldg(reinterpret_cast<const float2*>(sw + c0 + 2 * lane));   // O % 16 == 0
+      }
+      if (ok) ok = mbar_wait(afull, local & 1, kSiteGemmAccum);
+      ok = __all_sync(0xffffffffu, ok);
+      tc_fence_after();
+      const uint32_t tb = tmem + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(part * G::EpiCols);
+      uint32_t v[2][32];
+      tmem_ld_32x32b_x32(tb, v[0]);
+      tmem_ld_32x32b_x32(tb + 32, v[1]);
+      tmem_wait_ld();
+      // the accumulator is read out: hand it back to the MMA warp of the leader
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(aempty_leader);
+      if constexpr (!I32OUT) {
+        reinterpret_cast<float2*>(sws)[lane] = sw2;
+        __syncwarp();
+      }
+      float rmax = 0.f;
+      if (ok && y < N) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+          if (c0 + 32 * h < O) out.chunk(v[h], c0 + 32 * h, y, sa_r, sws + 32 * h, rmax);
+      }
+      // optional per-(row, 256-channel tile) maxima of |out|: the four warps
+      // of a lane quarter each hold a quarter of the tile's columns
+      if constexpr (ROWMAX && !I32OUT) {
+        float* slot = rmx + ((local & 1) * 4 + quad) * 4 * 32;
+        slot[part * 32 + lane] = rmax;
+        named_bar_sync(1 + quad, 128);
+        if (part == 0 && ok && row < N)
+          rowmax[static_cast<size_t>(row) * ntiles + n0 / kGemmBN] =
+              fmaxf(fmaxf(slot[lane], slot[32 + lane]), fmaxf(slot[64 + lane], slot[96 + lane]));
+      }
+    }
+    // the staging units must not be released while a store still reads them
+    if (lane == 0) bulk_wait_group_all();
+    __syncwarp();
+  }
+  tc_fence_before();
+  // Neither CTA of the pair may release its TMEM or shared memory while the
+  // other can still reach it.
+  cluster_sync();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, 512);
   }
 }
 
