@@ -668,10 +668,10 @@ def run_ours(args, rank: int, world: int, local_rank: int):
             "kernel_timing": "CUDA events around the boundary and GEMM launches of every %dth step "
                              "of the timed region (%d of %d steps)" % (EVERY, len(ev), Ksteps),
             "roofline": {
-                "kernel": "w4a4_gemm_kernel", "bound": "tensor",
+                "kernel": "w4a4_gemm_ta_kernel", "bound": "tensor",
                 "achieved": gemm_tops, "peak": int8_tops, "unit": "TFLOP/s",
                 "frac": gemm_tops / int8_tops,
-                "traffic": traffic_for("w4a4_gemm_kernels.cuh", "w4a4_gemm_kernel"),
+                "traffic": traffic_for("w4a4_gemm_kernels.cuh", "w4a4_gemm_ta_kernel"),
                 "peak_source": "%s bf16 burst %.1f TFLOP/s x %.0f (nominal "
                                "int8/bf16 dense ratio); integer ops counted "
                                "as 2 per multiply-add" % (src, bf16_tf,
