@@ -42,6 +42,9 @@ CASES = [
     ("tc_d8192_r128", 8192, 333, 128, 128, 0.1, 16, 100.0, "student_t3"),
     ("tc_d4096_r48", 4096, 520, 48, 64, 0.1, 8, 50.0, "normal"),
     ("tc_d1024_r128", 1024, 700, 128, 128, 0.5, 4, 50.0, "normal"),
+    # more token tiles (201) than SMs: the projection and re-projection grids
+    # take more than one wave
+    ("tc_d1024_r48_many_tiles", 1024, 25637, 48, 64, 0.1, 4, 50.0, "normal"),
     # rank 16 / 32 at D = 8192 (register-factor cluster plans) from 4096 tokens
     ("tc_d8192_r32", 8192, 4100, 32, 128, 0.1, 16, 100.0, "student_t3"),
     ("tc_d8192_r16", 8192, 4096, 16, 128, 0.1, 16, 100.0, "student_t3"),
