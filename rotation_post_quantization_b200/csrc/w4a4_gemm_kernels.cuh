@@ -551,6 +551,7 @@ struct GemmTaCfg {
   static_assert(BChunksPerThread * kTaProducerWarps * 32 == BNC * (kGemmBK / 32), "chunk split");
   static_assert(kTaProducerWarps == 4, "producer warp w widens the A rows of TMEM lane quarter w");
   static_assert(8 * (2 * US + 2 * PS + 2) + 4 <= 256, "barrier area");
+  static_assert(Smem <= 227 * 1024, "shared memory of one CTA");
 };
 
 // tmA: uint8 [N, K/2] box {64, 128}, 64-byte swizzle (row r's 16-byte piece j
