@@ -142,6 +142,13 @@ class ClockSampler(threading.Thread):
                 pass
             time.sleep(self.period)
 
+    def wait_first(self, limit_s: float = 2.0):
+        """Block until the thread has taken its first sample (the first NVML
+        query can take longer than a short timed region), at most limit_s."""
+        t_end = time.time() + limit_s
+        while self.ok and not self.samples and time.time() < t_end:
+            time.sleep(0.005)
+
     def summary(self, t0: float, t1: float):
         if not self.ok:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [],
@@ -489,7 +496,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
 
     sampler = ClockSampler(local_rank)
     sampler.start()
-    time.sleep(0.05)
+    sampler.wait_first()
 
     Ksteps = args.steps
     # per-kernel events on every EVERY-th step of the timed region (events

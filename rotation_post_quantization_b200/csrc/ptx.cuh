@@ -230,6 +230,21 @@ __device__ __forceinline__ void tma_store_2d(const void* tmap, int x, int y, uin
                : "memory");
 }
 
+// L2 policy that makes the lines it touches the first to be evicted.
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+// tma_store_2d with an L2 cache policy for the written lines.
+__device__ __forceinline__ void tma_store_2d_hint(const void* tmap, int x, int y, uint32_t src, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group.L2::cache_hint [%0, {%1, %2}], [%3], %4;" ::"l"(tmap),
+      "r"(x), "r"(y), "r"(src), "l"(policy)
+      : "memory");
+}
+
 __device__ __forceinline__ void bulk_commit_group() {
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }

@@ -135,9 +135,10 @@ struct GemmOut {
   uint32_t ubase;    // this warp's first staging unit (shared address)
   int lane, O;
   int unit;
+  uint64_t policy;   // the output is not read again by this kernel: its lines go first from L2
 
   __device__ __forceinline__ GemmOut(const CUtensorMap* tm, uint8_t* sm, uint32_t b, uint32_t ub, int ln, int o)
-      : tmO(tm), smem(sm), base(b), ubase(ub), lane(ln), O(o), unit(0) {}
+      : tmO(tm), smem(sm), base(b), ubase(ub), lane(ln), O(o), unit(0), policy(l2_policy_evict_first()) {}
 
   // Staging of one unit: begin() waits until the unit's previous tensor store
   // has read it and returns its generic address; the caller writes the
@@ -154,7 +155,7 @@ struct GemmOut {
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) {
-      tma_store_2d(tmO, x, y, ubase + static_cast<uint32_t>((unit % EB) * Unit));
+      tma_store_2d_hint(tmO, x, y, ubase + static_cast<uint32_t>((unit % EB) * Unit), policy);
       bulk_commit_group();
     }
     ++unit;
