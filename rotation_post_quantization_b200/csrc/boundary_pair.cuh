@@ -174,18 +174,22 @@ boundary_pair_kernel(const __grid_constant__ CUtensorMap tmR, const __grid_const
   // counted per barrier for the parity of the next wait.
   bool res_pend = false, x_pend0 = false, x_pend1 = false;
   uint32_t res_done = 0, x_done0 = 0, x_done1 = 0;
+  // residual and x are read once and h' is not read again by this launch:
+  // their L2 lines go first, so the codes and the next GEMM's weights stay
+  const uint64_t pol_ef = l2_policy_evict_first();
   auto issue_res = [&](int r) {
     if (lane == 0) mbar_arrive_expect_tx(rbar, NB * kPrBlockBytes);
     __syncwarp();
     if (lane < NB)
-      tma_load_2d(sRes + (b0 + lane) * kPrBlockBytes, &tmR, col0 + (b0 + lane) * 64, (cid + r * ncl) * T, rbar);
+      tma_load_2d_hint(sRes + (b0 + lane) * kPrBlockBytes, &tmR, col0 + (b0 + lane) * 64, (cid + r * ncl) * T, rbar,
+                       pol_ef);
     res_pend = true;
   };
   auto issue_x = [&](int r, int j) {   // block j of round r into slot j & 1
     const int s = j & 1;
     if (lane == s) {
       mbar_arrive_expect_tx(xbar(s), kPrBlockBytes);
-      tma_load_2d(sX + s * 8 * kPrBlockBytes, &tmX, col0 + (b0 + j) * 64, (cid + r * ncl) * T, xbar(s));
+      tma_load_2d_hint(sX + s * 8 * kPrBlockBytes, &tmX, col0 + (b0 + j) * 64, (cid + r * ncl) * T, xbar(s), pol_ef);
     }
     if (s) x_pend1 = true; else x_pend0 = true;
   };
@@ -381,7 +385,7 @@ boundary_pair_kernel(const __grid_constant__ CUtensorMap tmR, const __grid_const
               hp[0] = make_float4(hf[0].x, hf[0].y, hf[1].x, hf[1].y);
               hp[1] = make_float4(hf[2].x, hf[2].y, hf[3].x, hf[3].y);
             } else {
-              *reinterpret_cast<uint4*>(static_cast<bf16*>(h_out) + gi) = hv;
+              st_global_v4_hint(static_cast<bf16*>(h_out) + gi, hv, pol_ef);
             }
           }
         }
